@@ -1,0 +1,412 @@
+"""Benchmark of the MoC sparse-attention forward pass (one JSON line on rank 0).
+
+A step is one pass of the whole hot path over one scene: (1) pool keys,
+(2) route, (3) build query lists, (4) attend, (5) merge. Default workload:
+the eight-shot 180,512-token scene (B=1, H=24, d=128, k=3). Inputs are larger
+than L2 (3 x 1.1 GB), so no L2 flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--config eight|single|tiny|ragged|stress] [--k K]
+
+Under torchrun every rank runs its own independent scene (weak scaling: the
+per-GPU work is fixed); there is no collective on the data path. Times are
+CUDA-event device times, max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import moc_workloads as W  # noqa: E402
+
+METRIC = "MoC fwd tokens/s and selected-pair TFLOP/s (% bf16 peak) at 180k tokens"
+STAGES = ["pool", "route", "qlist", "attend", "merge"]
+LAUNCHES_PER_STEP = {"pool": 1, "route": 1, "qlist": 4, "attend": 1, "merge": 1}
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def workload(name: str, k):
+    wl = W.CONFIGS[name]()
+    return wl.with_k(k) if k is not None else wl
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi SM clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+def kernel_traffic():
+    """Per-launch DRAM bytes of the attend kernel from the committed ncu
+    summary, if it was taken on the current kernel source (else None)."""
+    src = os.path.join(ROOT, "chunk_routed_sparse_b200", "csrc", "k_attend_tc.cu")
+    if not os.path.exists(src):
+        src = os.path.join(ROOT, "chunk_routed_sparse_b200", "csrc", "k_attend_mma.cu")
+    summ = os.path.join(ROOT, "profiles", "attend_traffic.txt")
+    if not os.path.exists(summ):
+        return None
+    vals = {}
+    with open(summ) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                a, b = line.split(":", 1)
+                vals[a.strip()] = b.strip()
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if vals.get("source_sha256_16") != h or "dram_bytes_per_launch_full_scene" not in vals:
+        return None
+    return float(vals["dram_bytes_per_launch_full_scene"])
+
+
+def selected_pairs(layout_tables, wl, sel: torch.Tensor) -> int:
+    """Kept (query, key) pairs of the whole problem: anchor pairs from the
+    layout's group key counts plus the sizes of the selected chunks."""
+    grp, ar, ar_off = layout_tables
+    anchor = 0
+    for g in range(len(grp) // 2):
+        nq = grp[2 * g + 1] - grp[2 * g]
+        keys = sum(ar[2 * x + 1] - ar[2 * x] for x in range(ar_off[g], ar_off[g + 1]))
+        anchor += nq * keys
+    anchor *= wl.B * wl.H
+    ln = torch.tensor([s.length for s in wl.segments], dtype=torch.int64, device=sel.device)
+    routed = int(ln[sel[sel >= 0].long()].sum().item()) if sel.numel() else 0
+    return anchor + routed
+
+
+def run_ours(args):
+    import chunk_routed_sparse_b200 as moc
+
+    ws_, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if ws_ > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    wl = workload(args.config, args.k)
+    wl = wl.replace(seed=wl.seed + 1000 * rank)  # an independent scene per rank
+    B, H, L, d, k = wl.B, wl.H, wl.L, wl.d, wl.k
+    Qh, Kh, Vh = W.make_qkv(wl)
+    Qh, Kh, Vh = Qh.pin_memory(), Kh.pin_memory(), Vh.pin_memory()
+    dev = torch.device("cuda", local)
+    Q, K, V = (t.to(dev, non_blocking=False) for t in (Qh, Kh, Vh))
+    lay = moc.Layout.from_workload(wl, device=local)
+    kbar = torch.empty(B, H, lay.C, d, dtype=torch.float32, device=dev)
+    sel = torch.empty(B, H, L, k, dtype=torch.int32, device=dev)
+    ws = moc.workspace(lay, B, H, d, k, dev)
+    O = torch.empty_like(Q)
+    lse = torch.empty(B, H, L, dtype=torch.float32, device=dev)
+    scale = 1.0 / math.sqrt(d)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev: ev[0].record(stream)
+        moc.pool_keys(lay, K, out=kbar)
+        if ev: ev[1].record(stream)
+        if k > 0:
+            moc.route(lay, Q, kbar, k, wl.causal, out=sel)
+        if ev: ev[2].record(stream)
+        moc.build_qlists(lay, sel, B, H, k, ws)
+        if ev: ev[3].record(stream)
+        moc.attend_partials(lay, Q, K, V, k, ws, scale)
+        if ev: ev[4].record(stream)
+        moc.merge(lay, sel, k, ws, O, lse)
+        if ev: ev[5].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    moc.check_device_error(ws)
+    torch.cuda.synchronize()
+    pairs = selected_pairs((lay.table(1), lay.table(2), lay.table(3)), wl, sel)
+    flops = 4.0 * d * pairs
+
+    def barrier():
+        if ws_ > 1:
+            torch.distributed.barrier()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    stage_ms = {s: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
+                for j, s in enumerate(STAGES)}
+    moc.check_device_error(ws)
+
+    # end to end through the public API: pinned host inputs -> device -> result back
+    Oh = torch.empty_like(Qh).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(1, min(args.steps, 5))
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        Q.copy_(Qh, non_blocking=True)
+        K.copy_(Kh, non_blocking=True)
+        V.copy_(Vh, non_blocking=True)
+        step()
+        Oh.copy_(O, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+
+    if ws_ > 1:
+        t = torch.tensor([total_ms, e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms, e2e_ms = float(t[0]), float(t[1])
+
+    ms_per_step = total_ms / args.steps
+    tokens = B * L
+    peaks, peak_src = load_peaks()
+    att_s = stage_ms["attend"] / 1e3
+    achieved_tf = flops / att_s / 1e12
+    peak_tf = float(peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"]))
+    traffic = kernel_traffic()
+    dense_pairs = B * H * L * L
+    line = {
+        "metric": METRIC,
+        "value": ws_ * tokens / (ms_per_step / 1e3),
+        "unit": "tokens/s",
+        "n_gpus": ws_,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) + per-shot/per-frame mean offsets; no dataset)",
+        "config": {"workload": f"{wl.name}: B={B} H={H} L={L} d={d} k={k} chunks={lay.C} "
+                               f"anchor={wl.anchor} causal={wl.causal}",
+                   "tokens_per_step_per_gpu": tokens,
+                   "l2": "inputs larger than L2 (3 x %.2f GB), no flush" % (Q.numel() * 2 / 1e9),
+                   "parallelism": f"replicas x{ws_} (independent scenes, no collective)"},
+        "selected_pair_tflops_attend": achieved_tf,
+        "selected_pair_tflops_step": flops / (ms_per_step / 1e3) / 1e12,
+        "pct_bf16_peak_attend": 100.0 * achieved_tf / peak_tf,
+        "stage_ms": stage_ms,
+        "pruned_fraction": 1.0 - pairs / dense_pairs,
+        "kept_pairs": pairs,
+        "roofline": {"bound": "tensor", "kernel": "attend (4)", "achieved": achieved_tf,
+                     "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved_tf / peak_tf,
+                     "peak_kind": f"bf16_tflops_sustained ({peak_src})",
+                     "frac_of_burst": achieved_tf / float(peaks.get("bf16_tflops", 1590.0)),
+                     "traffic": traffic},
+        "hbm_kernels": hbm_fracs(stage_ms, B, H, L, lay.C, d, k, peaks),
+        "clocks": clk,
+        "e2e": {"value": ws_ * tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+                "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": 3 * Q.numel() * 2, "d2h_bytes_per_step": O.numel() * 2},
+        "gpu_launches": args.steps * sum(LAUNCHES_PER_STEP.values()),
+    }
+    if rank == 0 and ws_ == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, Qh, Kh, Vh, budget_s=args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws_ > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def hbm_fracs(stage_ms, B, H, L, C, d, k, peaks):
+    """Achieved GB/s of the HBM-bound kernels on their algorithmic bytes."""
+    hbm = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
+    BH = B * H
+    alg = {
+        "pool": BH * L * 2 * d + BH * C * d * 4,
+        "route": BH * L * 2 * d + BH * L * 4 * k,
+        "merge": BH * L * ((k + 1) * (4 * d + 4) + 4 * k + 2 * d + 4),
+    }
+    out = {}
+    for s, b in alg.items():
+        gbs = b / (stage_ms[s] / 1e3) / 1e9
+        out[s] = {"bytes": b, "GB/s": gbs, "frac_measured_hbm": gbs / hbm, "frac_8TBs": gbs / 8000.0}
+    return out
+
+
+def cpu_baseline(wl, Qh, Kh, Vh, budget_s: float = 20.0, rows_per_round: int = 64, seed: int = 0):
+    """The oracle as it stands, on this host's cores, on a bounded sample: one
+    head's pooling plus routing and attention of uniformly drawn query rows
+    until ~budget_s of work; scaled to tokens/s of the whole problem."""
+    import oracle
+
+    w1 = wl.replace(B=1, H=1)
+    q, kk, v = (t[0:1, 0:1].contiguous() for t in (Qh, Kh, Vh))
+    lay = oracle.Layout(w1)
+    t0 = time.perf_counter()
+    kbar = oracle.pool(w1, kk, lay)
+    t_pool = time.perf_counter() - t0
+    rng = np.random.default_rng(seed)
+    n, t_rows = 0, 0.0
+    while t_rows < budget_s:
+        rows = np.sort(rng.integers(0, lay.L, size=rows_per_round))
+        t1 = time.perf_counter()
+        rt = oracle.route(w1, q, kbar, rows=rows, lay=lay)
+        oracle.attend(w1, q, kk, v, rt["sel"], rows=rows, lay=lay)
+        t_rows += time.perf_counter() - t1
+        n += len(rows)
+    per_head = t_pool + t_rows * lay.L / n
+    value = wl.B * wl.L / (per_head * wl.B * wl.H)
+    return {"value": value, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"head (0,0): pool all {lay.C} chunks ({t_pool:.2f} s) + route/attend "
+                      f"{n} uniform query rows ({t_rows:.1f} s); extrapolated to {wl.B}x{wl.H} "
+                      f"heads x {lay.L} rows"}
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle, timed on this host's cores, each step a
+    bounded sample of the same workload (rank 0 only)."""
+    ws_, rank, _ = dist_env()
+    if rank != 0:
+        return
+    wl = workload(args.config, args.k)
+    Qh, Kh, Vh = W.make_qkv(wl, heads=[(0, 0)])
+    import oracle
+    w1 = wl.replace(B=1, H=1)
+    q, kk, v = (t[0:1, 0:1].contiguous() for t in (Qh, Kh, Vh))
+    lay = oracle.Layout(w1)
+    rng = np.random.default_rng(1)
+    rows_per_step = 48
+    t_pool = None
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        if t_pool is None:
+            kbar = oracle.pool(w1, kk, lay)
+            t_pool = time.perf_counter() - t0
+            t0 = time.perf_counter()
+        rows = np.sort(rng.integers(0, lay.L, size=rows_per_step))
+        rt = oracle.route(w1, q, kbar, rows=rows, lay=lay)
+        oracle.attend(w1, q, kk, v, rt["sel"], rows=rows, lay=lay)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    t_row = sum(times) / (len(times) * rows_per_step)
+    per_head = t_pool + t_row * lay.L
+    value = wl.B * wl.L / (per_head * wl.B * wl.H)
+    ms_per_step = per_head * wl.B * wl.H * 1e3
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": ws_, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{wl.name}: B={wl.B} H={wl.H} L={wl.L} d={wl.d} k={wl.k}"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.threads(),
+                             "kind": "oracle",
+                             "sample": f"per step {rows_per_step} uniform query rows of head (0,0) "
+                                       f"(route + attend), pooling once ({t_pool:.2f} s); "
+                                       f"extrapolated to the whole scene"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="eight", choices=sorted(W.CONFIGS))
+    ap.add_argument("--k", type=int, default=None)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,248 @@
+"""Mixture of Contexts (MoC) sparse-attention forward pass on B200 (sm_100a).
+
+Thin Python binding of the C ABI in ``include/moc.h`` (``libmoc.so``, built by
+``chunk_routed_sparse_b200/build.py``). It only marshals arguments: PyTorch
+provides device memory and the current CUDA stream, every step of the path
+runs in the library's CUDA kernels, and there is no CPU fallback - if the
+library is missing or a call fails, an exception is raised.
+
+Pipeline (pages: "Mixture of Contexts for Long Video Generation | Summary"
+§3.1-§3.3; the jxzklqfsx.com MoC write-up, "計算效率"):
+
+    layout = Layout(seg_len, seg_kind, seg_shot, seg_frame, anchor="shot")
+    kbar = pool_keys(layout, K)                  # (1) mean-pooled keys per chunk
+    sel = route(layout, Q, kbar, k, causal=True) # (2) top-k chunks per query
+    O, lse = attention_fwd(layout, Q, K, V, sel, k)  # (3) lists, (4) attend, (5) merge
+
+Q, K, V are bf16 CUDA tensors [B, H, L, d] (head-major, contiguous), d in {64, 128}.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoc.so")
+
+CAPTION, VIDEO = 0, 1
+ANCHOR = {"shot": 0, "local": 1, "chunk": 2}
+STATUS = {0: "ok", 1: "invalid argument", 2: "invalid layout description",
+          3: "workspace too small", 4: "CUDA error", 5: "device-side wait timed out",
+          6: "unsupported problem size", 7: "device-side consistency check failed"}
+
+
+class MocError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(status, status)} (status {status})")
+        self.status = status
+
+
+class _Desc(ctypes.Structure):
+    _fields_ = [("n_segments", ctypes.c_int32), ("seg_len", ctypes.c_void_p),
+                ("seg_kind", ctypes.c_void_p), ("seg_shot", ctypes.c_void_p),
+                ("seg_frame", ctypes.c_void_p), ("anchor_mode", ctypes.c_int32),
+                ("local_radius", ctypes.c_int32)]
+
+
+_lib = None
+
+# name -> (restype, argtypes); every symbol include/moc.h declares
+_I, _I64, _P, _F, _SZ = ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "moc_status_string": (ctypes.c_char_p, [_I]),
+    "moc_build_layout": (_I, [_P, _I, _P]),
+    "moc_layout_destroy": (None, [_P]),
+    "moc_layout_info": (_I, [_P, _P, _P, _P]),
+    "moc_layout_table": (_I, [_P, _I, _P, _I64, _P]),
+    "moc_pool_keys": (_I, [_P, _I, _I, _I, _P, _P, _P]),
+    "moc_route": (_I, [_P, _I, _I, _I, _P, _P, _I, _I, _P, _P]),
+    "moc_attention_workspace_bytes": (_SZ, [_P, _I, _I, _I, _I]),
+    "moc_build_qlists": (_I, [_P, _I, _I, _I, _P, _P, _SZ, _P]),
+    "moc_attend_partials": (_I, [_P, _I, _I, _I, _P, _P, _P, _I, _F, _P, _SZ, _P]),
+    "moc_merge": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _SZ, _P]),
+    "moc_attention_fwd": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _F, _P, _P, _P, _SZ, _P]),
+    "moc_check_device_error": (_I, [_P, _SZ, _P, _P]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoc.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: run chunk_routed_sparse_b200/build.py "
+                              "(there is no fallback implementation)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise MocError(status, where)
+
+
+def _stream() -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _i32(xs: Sequence[int]):
+    arr = (ctypes.c_int32 * len(xs))(*[int(x) for x in xs])
+    return arr
+
+
+class Layout:
+    """A scene's chunk tables (moc_build_layout), on the current CUDA device
+    by default, or host-only with ``device=-1`` (inspection only)."""
+
+    def __init__(self, seg_len, seg_kind, seg_shot, seg_frame, anchor: str = "shot",
+                 radius: int = 0, device: Optional[int] = None):
+        n = len(seg_len)
+        self._arrays = [_i32(seg_len), _i32(seg_kind), _i32(seg_shot), _i32(seg_frame)]
+        desc = _Desc(n, *[ctypes.cast(a, ctypes.c_void_p) for a in self._arrays],
+                     ANCHOR[anchor] if isinstance(anchor, str) else int(anchor), int(radius))
+        if device is None:
+            device = torch.cuda.current_device()
+        self.device = device
+        h = ctypes.c_void_p()
+        _check(lib().moc_build_layout(ctypes.byref(desc), int(device), ctypes.byref(h)),
+               "moc_build_layout")
+        self._h = h
+        L, C, S = ctypes.c_int64(), ctypes.c_int32(), ctypes.c_int32()
+        _check(lib().moc_layout_info(h, ctypes.byref(L), ctypes.byref(C), ctypes.byref(S)),
+               "moc_layout_info")
+        self.L, self.C, self.n_shots = L.value, C.value, S.value
+
+    @classmethod
+    def from_workload(cls, wl, device: Optional[int] = None) -> "Layout":
+        """From any object with seg_arrays(), ``anchor`` and ``radius``."""
+        ln, kind, shot, frame = wl.seg_arrays()
+        return cls(ln, kind, shot, frame, wl.anchor, wl.radius, device)
+
+    @property
+    def handle(self):
+        return self._h
+
+    def table(self, which: int):
+        n = ctypes.c_int64()
+        _check(lib().moc_layout_table(self._h, which, None, 0, ctypes.byref(n)), "moc_layout_table")
+        buf = (ctypes.c_int32 * max(n.value, 1))()
+        _check(lib().moc_layout_table(self._h, which, buf, n.value, ctypes.byref(n)),
+               "moc_layout_table")
+        return list(buf)[:n.value]
+
+    def workspace_bytes(self, B: int, H: int, d: int, k: int) -> int:
+        return int(lib().moc_attention_workspace_bytes(self._h, B, H, d, k))
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            lib().moc_layout_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def _dims(Q: torch.Tensor) -> Tuple[int, int, int, int]:
+    if Q.dim() != 4 or Q.dtype != torch.bfloat16 or not Q.is_cuda or not Q.is_contiguous():
+        raise ValueError("expected a contiguous bf16 CUDA tensor [B, H, L, d]")
+    return tuple(Q.shape)  # type: ignore
+
+
+def pool_keys(layout: Layout, K: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    B, H, L, d = _dims(K)
+    if out is None:
+        out = torch.empty(B, H, layout.C, d, dtype=torch.float32, device=K.device)
+    _check(lib().moc_pool_keys(layout.handle, B, H, d, _ptr(K), _ptr(out), _stream()),
+           "moc_pool_keys")
+    return out
+
+
+def route(layout: Layout, Q: torch.Tensor, kbar: torch.Tensor, k: int, causal: bool = True,
+          out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    B, H, L, d = _dims(Q)
+    if out is None:
+        out = torch.empty(B, H, L, k, dtype=torch.int32, device=Q.device)
+    _check(lib().moc_route(layout.handle, B, H, d, _ptr(Q), _ptr(kbar), k, int(bool(causal)),
+                           _ptr(out), _stream()), "moc_route")
+    return out
+
+
+def workspace(layout: Layout, B: int, H: int, d: int, k: int, device=None) -> torch.Tensor:
+    n = layout.workspace_bytes(B, H, d, k)
+    if n == 0:
+        raise ValueError("invalid problem for the workspace size query")
+    return torch.empty(n, dtype=torch.uint8, device=device or torch.cuda.current_device())
+
+
+def build_qlists(layout, sel, B, H, k, ws):
+    _check(lib().moc_build_qlists(layout.handle, B, H, k, _ptr(sel) if k > 0 else None, _ptr(ws),
+                                  ws.numel(), _stream()), "moc_build_qlists")
+
+
+def attend_partials(layout, Q, K, V, k, ws, scale=None):
+    B, H, L, d = _dims(Q)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    _check(lib().moc_attend_partials(layout.handle, B, H, d, _ptr(Q), _ptr(K), _ptr(V), k,
+                                     float(scale), _ptr(ws), ws.numel(), _stream()),
+           "moc_attend_partials")
+
+
+def merge(layout, sel, k, ws, O, lse=None):
+    B, H, L, d = _dims(O)
+    _check(lib().moc_merge(layout.handle, B, H, d, k, _ptr(sel) if k > 0 else None, _ptr(O),
+                           _ptr(lse), _ptr(ws), ws.numel(), _stream()), "moc_merge")
+
+
+def attention_fwd(layout: Layout, Q, K, V, sel, k: int, scale: Optional[float] = None,
+                  ws: Optional[torch.Tensor] = None, O: Optional[torch.Tensor] = None,
+                  lse: Optional[torch.Tensor] = None, want_lse: bool = True):
+    B, H, L, d = _dims(Q)
+    for t in (K, V):
+        if tuple(t.shape) != (B, H, L, d):
+            raise ValueError("Q, K, V shapes differ")
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if ws is None:
+        ws = workspace(layout, B, H, d, k, Q.device)
+    if O is None:
+        O = torch.empty_like(Q)
+    if lse is None and want_lse:
+        lse = torch.empty(B, H, L, dtype=torch.float32, device=Q.device)
+    _check(lib().moc_attention_fwd(layout.handle, B, H, d, _ptr(Q), _ptr(K), _ptr(V),
+                                   _ptr(sel) if k > 0 else None, k, float(scale), _ptr(O),
+                                   _ptr(lse), _ptr(ws), ws.numel(), _stream()),
+           "moc_attention_fwd")
+    return O, lse
+
+
+def forward(layout: Layout, Q, K, V, k: int, causal: bool = True, scale=None, ws=None):
+    """Pool -> route -> attention. Returns (O, lse, sel, kbar)."""
+    kbar = pool_keys(layout, K)
+    sel = route(layout, Q, kbar, k, causal) if k > 0 else \
+        torch.empty(Q.shape[0], Q.shape[1], Q.shape[2], 0, dtype=torch.int32, device=Q.device)
+    O, lse = attention_fwd(layout, Q, K, V, sel, k, scale=scale, ws=ws)
+    return O, lse, sel, kbar
+
+
+def check_device_error(ws: torch.Tensor) -> int:
+    """Read and clear the workspace's device error word (synchronises); returns
+    the detail code, raises MocError on a recorded device error."""
+    det = ctypes.c_int32()
+    st = lib().moc_check_device_error(_ptr(ws), ws.numel(), ctypes.byref(det), _stream())
+    _check(st, "device error word")
+    return det.value

@@ -1,0 +1,189 @@
+// C-ABI entry points: argument validation, workspace carve-up and kernel
+// launches. Every compute call is asynchronous on the caller's stream and
+// allocates nothing.
+#include <cstring>
+
+#include "moc_internal.h"
+
+namespace {
+
+constexpr size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+moc_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOC_OK : MOC_ERR_CUDA; }
+
+// Checks shared by the compute calls.
+moc_status check_common(const moc_layout* lay, int B, int H, int d, int k) {
+    if (!lay) return MOC_ERR_INVALID_ARG;
+    if (lay->device < 0 || !lay->dev_block) return MOC_ERR_INVALID_ARG;  // host-only layout
+    if (B < 0 || H < 0 || int64_t(B) * H > 65535) return MOC_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return MOC_ERR_INVALID_ARG;
+    if (k < 0 || k > moc::kMaxK) return MOC_ERR_INVALID_ARG;
+    const int64_t BH = int64_t(B) * H;
+    if (BH * lay->L * (k > 0 ? k : 1) >= (int64_t(1) << 31)) return MOC_ERR_UNSUPPORTED;
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) return MOC_ERR_CUDA;
+    if (cur != lay->device) return MOC_ERR_INVALID_ARG;
+    return MOC_OK;
+}
+
+}  // namespace
+
+namespace moc {
+
+WsPlan plan_workspace(const moc_layout* lay, int B, int H, int d, int k) {
+    WsPlan p;
+    const size_t BH = size_t(B) * H, L = size_t(lay->L), C = size_t(lay->C), S = size_t(k) + 1;
+    p.nblk = int((L + kQlistBlock - 1) / kQlistBlock);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off += align256(bytes);
+        return o;
+    };
+    p.hdr = take(64 * sizeof(int32_t));
+    p.blk_count = take(BH * size_t(p.nblk) * C * sizeof(int32_t));
+    p.qoff = take((BH * C + 1) * sizeof(int32_t));
+    p.tile_off = take((BH * C + 1) * sizeof(int32_t));
+    p.qlist = take(BH * L * size_t(k) * sizeof(int32_t));
+    p.lse_p = take(BH * L * S * sizeof(float));
+    p.o_p = take(BH * L * S * size_t(d) * sizeof(float));
+    p.total = off;
+    return p;
+}
+
+}  // namespace moc
+
+extern "C" const char* moc_status_string(moc_status s) {
+    switch (s) {
+        case MOC_OK: return "ok";
+        case MOC_ERR_INVALID_ARG: return "invalid argument";
+        case MOC_ERR_LAYOUT: return "invalid layout description";
+        case MOC_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case MOC_ERR_CUDA: return "CUDA error";
+        case MOC_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+        case MOC_ERR_UNSUPPORTED: return "unsupported problem size";
+        case MOC_ERR_DEVICE_CHECK: return "device-side consistency check failed";
+    }
+    return "unknown status";
+}
+
+extern "C" moc_status moc_pool_keys(const moc_layout* lay, int B, int H, int d, const void* K,
+                                    float* Kbar, moc_stream_t stream) {
+    moc_status st = check_common(lay, B, H, d, 0);
+    if (st != MOC_OK) return st;
+    if (B * H == 0) return MOC_OK;
+    if (!K || !Kbar || !aligned16(K) || !aligned16(Kbar)) return MOC_ERR_INVALID_ARG;
+    return cuda_status(moc::launch_pool(lay->dv, B * H, d, K, Kbar, (cudaStream_t)stream));
+}
+
+extern "C" moc_status moc_route(const moc_layout* lay, int B, int H, int d, const void* Q,
+                                const float* Kbar, int k, int causal, int32_t* sel,
+                                moc_stream_t stream) {
+    moc_status st = check_common(lay, B, H, d, k);
+    if (st != MOC_OK) return st;
+    if (B * H == 0 || k == 0) return MOC_OK;
+    if (!Q || !Kbar || !sel || !aligned16(Q) || !aligned16(Kbar) ||
+        (reinterpret_cast<uintptr_t>(sel) & 3))
+        return MOC_ERR_INVALID_ARG;
+    return cuda_status(moc::launch_route(lay->dv, B * H, lay->total_rtiles, d, Q, Kbar, k,
+                                         causal ? 1 : 0, sel, (cudaStream_t)stream));
+}
+
+extern "C" size_t moc_attention_workspace_bytes(const moc_layout* lay, int B, int H, int d, int k) {
+    if (!lay || B < 0 || H < 0 || (d != 64 && d != 128) || k < 0 || k > moc::kMaxK) return 0;
+    return moc::plan_workspace(lay, B, H, d, k).total;
+}
+
+namespace {
+
+moc_status check_ws(const moc_layout* lay, int B, int H, int d, int k, void* ws, size_t ws_bytes,
+                    moc::WsPlan* p) {
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return MOC_ERR_INVALID_ARG;
+    *p = moc::plan_workspace(lay, B, H, d, k);
+    if (ws_bytes < p->total) return MOC_ERR_WORKSPACE_TOO_SMALL;
+    return MOC_OK;
+}
+
+}  // namespace
+
+extern "C" moc_status moc_build_qlists(const moc_layout* lay, int B, int H, int k,
+                                       const int32_t* sel, void* ws, size_t ws_bytes,
+                                       moc_stream_t stream) {
+    moc_status st = check_common(lay, B, H, 128, k);
+    if (st != MOC_OK) return st;
+    if (B * H == 0) return MOC_OK;
+    moc::WsPlan p;
+    // the query lists do not depend on d; plan with the smallest d for the check
+    if ((st = check_ws(lay, B, H, 64, k, ws, ws_bytes, &p)) != MOC_OK) return st;
+    if (k > 0 && (!sel || (reinterpret_cast<uintptr_t>(sel) & 3))) return MOC_ERR_INVALID_ARG;
+    return cuda_status(moc::launch_qlists(lay->dv, B * H, k, sel, static_cast<char*>(ws), p,
+                                          (cudaStream_t)stream));
+}
+
+extern "C" moc_status moc_attend_partials(const moc_layout* lay, int B, int H, int d, const void* Q,
+                                          const void* K, const void* V, int k, float scale,
+                                          void* ws, size_t ws_bytes, moc_stream_t stream) {
+    moc_status st = check_common(lay, B, H, d, k);
+    if (st != MOC_OK) return st;
+    if (B * H == 0) return MOC_OK;
+    moc::WsPlan p;
+    if ((st = check_ws(lay, B, H, d, k, ws, ws_bytes, &p)) != MOC_OK) return st;
+    if (!Q || !K || !V || !aligned16(Q) || !aligned16(K) || !aligned16(V)) return MOC_ERR_INVALID_ARG;
+    if (!(scale > 0.0f) || scale != scale) return MOC_ERR_INVALID_ARG;
+    const int64_t n_anchor = int64_t(B) * H * lay->total_atiles;
+    return cuda_status(moc::launch_attend(lay->dv, B * H, d, Q, K, V, k, scale, n_anchor,
+                                          static_cast<char*>(ws), p, (cudaStream_t)stream));
+}
+
+extern "C" moc_status moc_merge(const moc_layout* lay, int B, int H, int d, int k,
+                                const int32_t* sel, void* O, float* lse, void* ws, size_t ws_bytes,
+                                moc_stream_t stream) {
+    moc_status st = check_common(lay, B, H, d, k);
+    if (st != MOC_OK) return st;
+    if (B * H == 0) return MOC_OK;
+    moc::WsPlan p;
+    if ((st = check_ws(lay, B, H, d, k, ws, ws_bytes, &p)) != MOC_OK) return st;
+    if (!O || !aligned16(O) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3))) return MOC_ERR_INVALID_ARG;
+    if (k > 0 && (!sel || (reinterpret_cast<uintptr_t>(sel) & 3))) return MOC_ERR_INVALID_ARG;
+    return cuda_status(moc::launch_merge(B * H, int(lay->L), d, k, sel, O, lse,
+                                         static_cast<const char*>(ws), p, (cudaStream_t)stream));
+}
+
+extern "C" moc_status moc_attention_fwd(const moc_layout* lay, int B, int H, int d, const void* Q,
+                                        const void* K, const void* V, const int32_t* sel, int k,
+                                        float scale, void* O, float* lse, void* ws,
+                                        size_t ws_bytes, moc_stream_t stream) {
+    moc_status st = check_common(lay, B, H, d, k);
+    if (st != MOC_OK) return st;
+    if (B * H == 0) return MOC_OK;
+    moc::WsPlan p;
+    if ((st = check_ws(lay, B, H, d, k, ws, ws_bytes, &p)) != MOC_OK) return st;
+    if (!Q || !K || !V || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+        return MOC_ERR_INVALID_ARG;
+    if (k > 0 && (!sel || (reinterpret_cast<uintptr_t>(sel) & 3))) return MOC_ERR_INVALID_ARG;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3)) return MOC_ERR_INVALID_ARG;
+    if (!(scale > 0.0f) || scale != scale) return MOC_ERR_INVALID_ARG;
+    if ((st = moc_build_qlists(lay, B, H, k, sel, ws, ws_bytes, stream)) != MOC_OK) return st;
+    if ((st = moc_attend_partials(lay, B, H, d, Q, K, V, k, scale, ws, ws_bytes, stream)) != MOC_OK)
+        return st;
+    return moc_merge(lay, B, H, d, k, sel, O, lse, ws, ws_bytes, stream);
+}
+
+extern "C" moc_status moc_check_device_error(void* ws, size_t ws_bytes, int32_t* detail,
+                                             moc_stream_t stream) {
+    if (!ws || ws_bytes < 64 * sizeof(int32_t)) return MOC_ERR_INVALID_ARG;
+    int32_t h[2] = {0, 0};
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(h, ws, sizeof h, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOC_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOC_ERR_CUDA;
+    if (detail) *detail = h[1];
+    if (h[0] != moc::ERR_NONE) {
+        if (cudaMemsetAsync(ws, 0, 2 * sizeof(int32_t), s) != cudaSuccess) return MOC_ERR_CUDA;
+        if (cudaStreamSynchronize(s) != cudaSuccess) return MOC_ERR_CUDA;
+    }
+    if (h[0] == moc::ERR_TIMEOUT) return MOC_ERR_DEVICE_TIMEOUT;
+    if (h[0] == moc::ERR_CHECK) return MOC_ERR_DEVICE_CHECK;
+    return MOC_OK;
+}

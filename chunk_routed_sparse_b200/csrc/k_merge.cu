@@ -1,0 +1,90 @@
+// (5) Log-sum-exp merge of each query's partial attention outputs.
+//
+// The attention of "Mixture of Contexts for Long Video Generation | Summary"
+// §3.1 runs over Omega(q) = anchors + selected chunks. The attend kernel
+// computes it in disjoint parts (slot 0: anchors; slot 1+x: the chunk in
+// sel[x]), each normalised with its own log-sum-exp l_j. Softmax over a
+// disjoint union recombines exactly:
+//   M = max_j l_j,  w_j = exp(l_j - M),  O = sum_j w_j O_j / sum_j w_j,
+//   lse = M + log sum_j w_j.
+// One warp per (b*h, query); slots in fixed order -> deterministic.
+// HBM-bound: reads (1+k)*(4d+4) bytes and writes 2d+4 bytes per query.
+#include "common.cuh"
+
+namespace moc {
+namespace {
+
+template <int D>
+__global__ void __launch_bounds__(256) merge_kernel(int64_t rows, int L, int k,
+                                                    const int32_t* __restrict__ sel,
+                                                    const float* __restrict__ lse_p,
+                                                    const float* __restrict__ o_p,
+                                                    __nv_bfloat16* __restrict__ O,
+                                                    float* __restrict__ lse) {
+    constexpr int PER = D / 32;  // output columns per lane
+    const int lane = threadIdx.x & 31;
+    const int S = k + 1;
+    for (int64_t row = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; row < rows;
+         row += (int64_t(gridDim.x) * blockDim.x) >> 5) {
+        bool valid = false;
+        float l = -INFINITY;
+        if (lane < S) {
+            valid = (lane == 0) || (sel[row * k + lane - 1] >= 0);
+            if (valid) l = lse_p[row * S + lane];
+        }
+        float m = l;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const float w = valid ? expf(l - m) : 0.f;
+        float z = w;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+        const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+        float acc[PER];
+#pragma unroll
+        for (int x = 0; x < PER; ++x) acc[x] = 0.f;
+        const float* op = o_p + size_t(row) * S * D + lane * PER;
+        for (unsigned mm = vmask; mm; mm &= mm - 1) {
+            const int j = __ffs(mm) - 1;
+            const float wj = __shfl_sync(0xffffffffu, w, j) / z;
+            if (PER == 4) {
+                const float4 v = *reinterpret_cast<const float4*>(op + size_t(j) * D);
+                acc[0] += wj * v.x; acc[1] += wj * v.y; acc[2] += wj * v.z; acc[3] += wj * v.w;
+            } else {
+                const float2 v = *reinterpret_cast<const float2*>(op + size_t(j) * D);
+                acc[0] += wj * v.x; acc[1] += wj * v.y;
+            }
+        }
+        __nv_bfloat16* orow = O + size_t(row) * D + lane * PER;
+        if (PER == 4) {
+            uint2 pk = make_uint2(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]));
+            *reinterpret_cast<uint2*>(orow) = pk;
+        } else {
+            *reinterpret_cast<uint32_t*>(orow) = pack_bf16(acc[0], acc[1]);
+        }
+        if (lse && lane == 0) lse[row] = m + logf(z);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_merge(int BH, int L, int d, int k, const int32_t* sel, void* O, float* lse,
+                         const char* ws, const WsPlan& p, cudaStream_t s) {
+    const int64_t rows = int64_t(BH) * L;
+    const float* lse_p = reinterpret_cast<const float*>(ws + p.lse_p);
+    const float* o_p = reinterpret_cast<const float*>(ws + p.o_p);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t want = (rows + 7) / 8;
+    const int grid = int(want < int64_t(sms) * 16 ? want : int64_t(sms) * 16);
+    if (d == 128)
+        merge_kernel<128><<<grid, 256, 0, s>>>(rows, L, k, sel, lse_p, o_p,
+                                               static_cast<__nv_bfloat16*>(O), lse);
+    else
+        merge_kernel<64><<<grid, 256, 0, s>>>(rows, L, k, sel, lse_p, o_p,
+                                              static_cast<__nv_bfloat16*>(O), lse);
+    return cudaGetLastError();
+}
+
+}  // namespace moc

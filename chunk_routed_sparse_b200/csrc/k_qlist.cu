@@ -1,0 +1,164 @@
+// (3) Query-list builder: invert the per-query selections into per-chunk
+// query lists (count -> exclusive prefix sum -> ordered scatter).
+//
+// This replaces the "pack every (query, key) group into one variable-length
+// attention call" step of the jxzklqfsx.com MoC write-up ("計算效率"): the
+// attention kernel walks chunk-major work items, each a chunk's keys against
+// up to 128 of the queries that selected it.
+//
+// Entries are (query << 5 | slot), slot = position in sel. Every list is
+// sorted by query: each block owns kQlistBlock consecutive queries and one
+// warp walks them in order, ranking equal chunk ids inside a 32-entry step
+// with __match_any_sync, so the output is deterministic.
+#include "common.cuh"
+
+namespace moc {
+namespace {
+
+// blk_count[bh][blk][c] = entries of chunk c among the block's queries
+__global__ void __launch_bounds__(32) qlist_count(int L, int C, int k, int nblk,
+                                                  const int32_t* __restrict__ sel,
+                                                  int32_t* __restrict__ blk_count,
+                                                  int32_t* __restrict__ hdr) {
+    extern __shared__ int32_t cnt[];
+    const int blk = blockIdx.x, bh = blockIdx.y, lane = threadIdx.x;
+    for (int c = lane; c < C; c += 32) cnt[c] = 0;
+    __syncwarp();
+    const int q0 = blk * kQlistBlock, q1 = min(L, q0 + kQlistBlock);
+    const int32_t* s = sel + (size_t(bh) * L) * k;
+    for (int64_t e = int64_t(q0) * k + lane; e < int64_t(q1) * k; e += 32) {
+        const int c = s[e];
+        if (c >= C) set_error(hdr, ERR_CHECK, 3);  // not a chunk id: entry ignored
+        else if (c >= 0) atomicAdd(&cnt[c], 1);
+    }
+    __syncwarp();
+    int32_t* out = blk_count + (size_t(bh) * nblk + blk) * C;
+    for (int c = lane; c < C; c += 32) out[c] = cnt[c];
+}
+
+// Per (bh): blk_count -> exclusive offsets of each block within each chunk's
+// list (in place); qoff[bh*C + c] <- list length, tile_off[bh*C + c] <- tiles.
+__global__ void __launch_bounds__(256) qlist_scan_blocks(int C, int nblk,
+                                                         int32_t* __restrict__ blk_count,
+                                                         int32_t* __restrict__ qlen,
+                                                         int32_t* __restrict__ ntile) {
+    const int bh = blockIdx.x;
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+        int32_t run = 0;
+        int32_t* p = blk_count + size_t(bh) * nblk * C + c;
+        for (int b = 0; b < nblk; ++b) {
+            const int32_t v = p[size_t(b) * C];
+            p[size_t(b) * C] = run;
+            run += v;
+        }
+        qlen[size_t(bh) * C + c] = run;
+        ntile[size_t(bh) * C + c] = (run + kQTile - 1) / kQTile;
+    }
+}
+
+// In-place exclusive scan of two int32 arrays of n values (+ total at [n]),
+// one CTA of 1024 threads.
+__global__ void __launch_bounds__(1024) qlist_scan_global(int64_t n, int32_t* __restrict__ a,
+                                                          int32_t* __restrict__ b) {
+    __shared__ int32_t wa[32], wb[32];
+    __shared__ int32_t carry_a, carry_b;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) carry_a = carry_b = 0;
+    __syncthreads();
+    for (int64_t base = 0; base < n; base += 1024) {
+        const int64_t i = base + tid;
+        const int32_t va = (i < n) ? a[i] : 0, vb = (i < n) ? b[i] : 0;
+        int32_t xa = va, xb = vb;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t ya = __shfl_up_sync(0xffffffffu, xa, o), yb = __shfl_up_sync(0xffffffffu, xb, o);
+            if (lane >= o) { xa += ya; xb += yb; }
+        }
+        if (lane == 31) { wa[warp] = xa; wb[warp] = xb; }
+        __syncthreads();
+        if (warp == 0) {
+            int32_t sa = wa[lane], sb = wb[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int32_t ya = __shfl_up_sync(0xffffffffu, sa, o), yb = __shfl_up_sync(0xffffffffu, sb, o);
+                if (lane >= o) { sa += ya; sb += yb; }
+            }
+            wa[lane] = sa;
+            wb[lane] = sb;
+        }
+        __syncthreads();
+        const int32_t pa = carry_a + (warp ? wa[warp - 1] : 0) + xa - va;
+        const int32_t pb = carry_b + (warp ? wb[warp - 1] : 0) + xb - vb;
+        if (i < n) { a[i] = pa; b[i] = pb; }
+        __syncthreads();
+        if (tid == 1023) { carry_a = pa + va; carry_b = pb + vb; }
+        __syncthreads();
+    }
+    if (tid == 0) { a[n] = carry_a; b[n] = carry_b; }
+}
+
+__global__ void __launch_bounds__(32) qlist_scatter(int L, int C, int k, int nblk,
+                                                    const int32_t* __restrict__ sel,
+                                                    const int32_t* __restrict__ blk_count,
+                                                    const int32_t* __restrict__ qoff,
+                                                    int32_t* __restrict__ qlist) {
+    extern __shared__ int32_t cur[];
+    const int blk = blockIdx.x, bh = blockIdx.y, lane = threadIdx.x;
+    const int32_t* bc = blk_count + (size_t(bh) * nblk + blk) * C;
+    const int32_t* qo = qoff + size_t(bh) * C;
+    for (int c = lane; c < C; c += 32) cur[c] = qo[c] + bc[c];
+    __syncwarp();
+    const int q0 = blk * kQlistBlock, q1 = min(L, q0 + kQlistBlock);
+    const int32_t* s = sel + (size_t(bh) * L) * k;
+    const unsigned lt = (1u << lane) - 1u;
+    for (int64_t e0 = int64_t(q0) * k; e0 < int64_t(q1) * k; e0 += 32) {
+        const int64_t e = e0 + lane;
+        int c = (e < int64_t(q1) * k) ? s[e] : -1;
+        if (c >= C) c = -1;  // reported by qlist_count
+        const unsigned peers = __match_any_sync(0xffffffffu, c);
+        const int rank = __popc(peers & lt);
+        const int base = (c >= 0) ? cur[c] : 0;
+        __syncwarp();
+        if (c >= 0) {
+            const int q = int(e / k), slot = int(e % k);
+            qlist[base + rank] = (q << 5) | slot;
+            if (rank == 0) cur[c] = base + __popc(peers);
+        }
+        __syncwarp();
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_qlists(const DevLayout& dv, int BH, int k, const int32_t* sel, char* ws,
+                          const WsPlan& p, cudaStream_t s) {
+    int32_t* hdr = reinterpret_cast<int32_t*>(ws + p.hdr);
+    cudaError_t e = cudaMemsetAsync(hdr, 0, 4 * sizeof(int32_t), s);
+    if (e != cudaSuccess) return e;
+    int32_t* blk_count = reinterpret_cast<int32_t*>(ws + p.blk_count);
+    int32_t* qoff = reinterpret_cast<int32_t*>(ws + p.qoff);
+    int32_t* tile_off = reinterpret_cast<int32_t*>(ws + p.tile_off);
+    int32_t* qlist = reinterpret_cast<int32_t*>(ws + p.qlist);
+    const int64_t n = int64_t(BH) * dv.C;
+    if (k == 0) {  // no routed work: empty lists
+        e = cudaMemsetAsync(qoff, 0, size_t(n + 1) * sizeof(int32_t), s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(tile_off, 0, size_t(n + 1) * sizeof(int32_t), s);
+        return e;
+    }
+    if (BH > 65535) return cudaErrorInvalidValue;
+    const size_t smem = size_t(dv.C) * sizeof(int32_t);
+    if (smem > 48 * 1024) {
+        e = cudaFuncSetAttribute(qlist_count, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(qlist_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return e;
+    }
+    dim3 grid(p.nblk, BH);
+    qlist_count<<<grid, 32, smem, s>>>(dv.L, dv.C, k, p.nblk, sel, blk_count, hdr);
+    qlist_scan_blocks<<<BH, 256, 0, s>>>(dv.C, p.nblk, blk_count, qoff, tile_off);
+    qlist_scan_global<<<1, 1024, 0, s>>>(n, qoff, tile_off);
+    qlist_scatter<<<grid, 32, smem, s>>>(dv.L, dv.C, k, p.nblk, sel, blk_count, qoff, qlist);
+    return cudaGetLastError();
+}
+
+}  // namespace moc

@@ -1,0 +1,84 @@
+// Internal declarations shared by the C-ABI glue and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "moc.h"
+
+namespace moc {
+
+constexpr int kQTile = 128;       // query rows per router / attention work item
+constexpr int kMaxK = 31;         // top-k limit: 1+k partial slots fit one warp
+constexpr int kMaxChunks = 16384; // chunk limit (query-list counters live in shared memory)
+constexpr int kQlistBlock = 1024; // queries per block of the query-list builder
+
+// Read-only view of a layout's device tables, passed to kernels by value.
+struct DevLayout {
+    int32_t L, C, G;
+    const int32_t* chunk_off;    // [C+1] token offset of every chunk
+    const int32_t* grp_q0;       // [G] first token of the group
+    const int32_t* grp_q1;       // [G] one past the last token
+    const int32_t* grp_kind;     // [G] MOC_CAPTION / MOC_VIDEO
+    const int32_t* ar_off;       // [G+1] offsets into ar
+    const int32_t* ar;           // anchor key ranges, (start, end) pairs
+    const int32_t* cand_off;     // [G+1] offsets into cand
+    const int32_t* cand;         // candidate chunk ids, ascending, per group
+    const int32_t* cand_ncausal; // [G] length of the causal prefix of the list
+    const int32_t* rtile_off;    // [G+1] prefix of router tiles (kQTile queries) per group
+    const int32_t* atile_off;    // [G+1] prefix of anchor tiles, groups in a_order
+    const int32_t* a_order;      // [G] groups by descending anchor keys per tile
+};
+
+}  // namespace moc
+
+struct moc_layout {
+    int device = -1;
+    int64_t L = 0;
+    int32_t C = 0, G = 0, n_shots = 0;
+    int32_t max_cand = 0;       // largest candidate list of any group
+    int64_t total_rtiles = 0;   // router tiles per (b, h)
+    int64_t total_atiles = 0;   // anchor tiles per (b, h)
+    std::vector<int32_t> chunk_off, kind, shot, frame;
+    std::vector<int32_t> grp_q0, grp_q1, grp_kind, ar_off, ar, cand_off, cand, cand_ncausal;
+    std::vector<int32_t> rtile_off, atile_off, a_order;
+    std::vector<int64_t> grp_keys;  // anchor keys of each group
+    void* dev_block = nullptr;
+    moc::DevLayout dv{};
+};
+
+namespace moc {
+
+// Workspace carve-up of moc_attention_fwd (all offsets 256-byte aligned).
+struct WsPlan {
+    size_t hdr = 0;        // int32[64]: [0] error code, [1] detail, [2] work counter
+    size_t blk_count = 0;  // int32 [BH][nblk][C]
+    size_t qoff = 0;       // int32 [BH*C + 1] global start of every list
+    size_t tile_off = 0;   // int32 [BH*C + 1] prefix of routed tiles
+    size_t qlist = 0;      // int32 [BH*L*k] entries (query << 5 | slot)
+    size_t lse_p = 0;      // fp32 [BH][L][1+k]
+    size_t o_p = 0;        // fp32 [BH][L][1+k][d]
+    size_t total = 0;
+    int nblk = 0;
+};
+WsPlan plan_workspace(const moc_layout* lay, int B, int H, int d, int k);
+
+enum { HDR_ERR = 0, HDR_DETAIL = 1, HDR_WORK = 2 };
+enum { ERR_NONE = 0, ERR_TIMEOUT = 1, ERR_CHECK = 2 };
+
+// Kernel launchers (return cudaGetLastError() of the launch).
+cudaError_t launch_pool(const DevLayout& dv, int BH, int d, const void* K, float* Kbar,
+                        cudaStream_t s);
+cudaError_t launch_route(const DevLayout& dv, int BH, int64_t rtiles, int d, const void* Q,
+                         const float* Kbar, int k, int causal, int32_t* sel, cudaStream_t s);
+cudaError_t launch_qlists(const DevLayout& dv, int BH, int k, const int32_t* sel, char* ws,
+                          const WsPlan& p, cudaStream_t s);
+cudaError_t launch_attend(const DevLayout& dv, int BH, int d, const void* Q, const void* K,
+                          const void* V, int k, float scale, int64_t n_anchor_items, char* ws,
+                          const WsPlan& p, cudaStream_t s);
+cudaError_t launch_merge(int BH, int L, int d, int k, const int32_t* sel, void* O, float* lse,
+                         const char* ws, const WsPlan& p, cudaStream_t s);
+
+}  // namespace moc

@@ -1,0 +1,183 @@
+/*
+ * moc.h - C ABI of the Mixture of Contexts (MoC) sparse-attention forward pass
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The method (pages: "Mixture of Contexts for Long Video Generation | Summary",
+ * §3.1-§3.3; the jxzklqfsx.com MoC write-up, sections "內容對齊的塊劃分",
+ * "固定的跨模態選擇", "固定的鏡頭內選擇", "稀疏 MoC 中的因果性", "計算效率"):
+ * the flattened text+video token stream is cut into content-aligned chunks
+ * (caption segments and video frames or sub-frames). Keys are mean-pooled per
+ * chunk. Every video query scores its candidate chunks by the dot product with
+ * the pooled keys and keeps the top-k; candidates are the video chunks that are
+ * not mandatory for it, restricted to strictly earlier chunks under the causal
+ * routing mask. Mandatory anchors (every caption token plus the query's own
+ * shot, local frame window or own chunk) are always attended. Exact softmax
+ * attention then runs over the union of anchors and selected chunks. Caption
+ * queries attend densely to every token of the sample.
+ *
+ * Conventions shared by every call:
+ *  - Tensors are head-major, contiguous: Q, K, V and O are bf16 [B][H][L][d];
+ *    d is 64 or 128. Device pointers must be 16-byte aligned.
+ *  - The caller owns every device buffer (inputs, outputs, workspace). The
+ *    library allocates device memory only inside moc_build_layout (its tables,
+ *    freed by moc_layout_destroy); no hot-path call allocates.
+ *  - Compute calls are asynchronous on the given stream and return after
+ *    enqueueing. Argument errors are returned before anything is enqueued;
+ *    a launch failure returns MOC_ERR_CUDA. No call throws across the ABI.
+ *  - Limits: 1 <= C <= 16384 chunks, L < 2^26, B*H <= 65535, B*H*L*max(k,1) < 2^31,
+ *    0 <= k <= 31, every chunk non-empty.
+ */
+#ifndef MOC_H
+#define MOC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream handle (the same object as cudaStream_t / CUstream). */
+struct CUstream_st;
+typedef struct CUstream_st* moc_stream_t;
+
+typedef enum {
+    MOC_OK = 0,
+    MOC_ERR_INVALID_ARG = 1,         /* null/misaligned pointer, bad size, bad k or d */
+    MOC_ERR_LAYOUT = 2,              /* inconsistent segment description */
+    MOC_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes < moc_attention_workspace_bytes(...) */
+    MOC_ERR_CUDA = 4,                /* a CUDA runtime call or launch failed */
+    MOC_ERR_DEVICE_TIMEOUT = 5,      /* a bounded device-side wait gave up */
+    MOC_ERR_UNSUPPORTED = 6,         /* valid request outside what this build handles */
+    MOC_ERR_DEVICE_CHECK = 7         /* a device-side consistency check failed */
+} moc_status;
+
+/* Segment kinds and anchor modes of moc_layout_desc. */
+enum { MOC_CAPTION = 0, MOC_VIDEO = 1 };
+enum {
+    MOC_ANCHOR_SHOT = 0,  /* every video chunk of the query's shot (multi-shot scenes) */
+    MOC_ANCHOR_LOCAL = 1, /* video chunks of the query's shot within +-local_radius frames */
+    MOC_ANCHOR_CHUNK = 2  /* the query's own chunk only */
+};
+
+/* Host-memory description of one scene's token stream, in stream order
+ * (content-aligned chunking: "內容對齊的塊劃分" of the jxzklqfsx.com write-up;
+ * the boundary tables of its "計算效率" section). Each segment is one chunk.
+ *   seg_len[i]   token count (> 0) of segment i;
+ *   seg_kind[i]  MOC_CAPTION or MOC_VIDEO;
+ *   seg_shot[i]  shot id of a video segment (informational for captions);
+ *   seg_frame[i] frame index of a video segment within its shot; sub-chunks
+ *                of one frame repeat it.
+ * Video segments of one shot must be contiguous in the stream with frame
+ * indices non-decreasing. The arrays are read during moc_build_layout only. */
+typedef struct {
+    int32_t n_segments;
+    const int32_t* seg_len;
+    const int32_t* seg_kind;
+    const int32_t* seg_shot;
+    const int32_t* seg_frame;
+    int32_t anchor_mode;   /* MOC_ANCHOR_* */
+    int32_t local_radius;  /* frames, for MOC_ANCHOR_LOCAL (>= 0) */
+} moc_layout_desc;
+
+typedef struct moc_layout moc_layout; /* opaque */
+
+/* Text of a status code (static storage). */
+const char* moc_status_string(moc_status s);
+
+/* Build the chunk tables of a scene: chunk offsets, chunk -> shot/frame/kind,
+ * query groups (runs of chunks sharing one anchor set), per-group anchor key
+ * ranges and candidate chunk lists ("計算效率": boundary tagging and prefix-sum
+ * tables; the pre-routing mask that keeps mandatory chunks out of top-k).
+ * device >= 0: the tables are also copied to that CUDA device (allocated here,
+ * freed by moc_layout_destroy); device == -1: host-only layout, usable with the
+ * query calls below but rejected by every compute call.
+ * On success *out owns the layout. On error *out is set to NULL. */
+moc_status moc_build_layout(const moc_layout_desc* desc, int device, moc_layout** out);
+
+/* Free a layout and its device tables (NULL is a no-op). Not stream-ordered:
+ * call it only when no launched work still uses the layout. */
+void moc_layout_destroy(moc_layout* layout);
+
+/* Sizes of a built layout: tokens L, chunks C, distinct shots (any may be NULL). */
+moc_status moc_layout_info(const moc_layout* layout, int64_t* L, int32_t* C, int32_t* n_shots);
+
+/* Host-side copy of one layout table, for inspection and tests.
+ * which: 0 chunk_off[C+1], 1 group token range (q0,q1)[G][2],
+ *        2 group anchor key ranges as (start,end) pairs in group order,
+ *        3 anchor range offsets per group [G+1], 4 candidate chunk ids in
+ *        group order, 5 candidate offsets per group [G+1],
+ *        6 causal candidate count per group [G].
+ * Writes min(count, cap) int32 values to out (may be NULL with cap 0) and
+ * the full count to *count. */
+moc_status moc_layout_table(const moc_layout* layout, int which, int32_t* out, int64_t cap,
+                            int64_t* count);
+
+/* (1) Segmented mean pool of keys ("計算效率": segment_reduce mean pooling;
+ * Summary §3.1: the chunk descriptor is the mean of the chunk's keys):
+ *   Kbar[b][h][c][e] = (1/n_c) * sum_{t in chunk c} K[b][h][t][e],
+ * accumulated in fp32 from bf16. K: device bf16 [B][H][L][d]; Kbar: device
+ * fp32 [B][H][C][d], 16-byte aligned. Deterministic. */
+moc_status moc_pool_keys(const moc_layout* layout, int B, int H, int d, const void* K,
+                         float* Kbar, moc_stream_t stream);
+
+/* (2) Routing (Summary §3.1 top-k by dot product with the pooled key; §3.2
+ * causal mask j < i before top-k; "計算效率": mandatory chunks excluded from
+ * the candidates). For every video query t of chunk i, candidates are the
+ * video chunks j that are not mandatory for it, and with causal != 0 only
+ * those with j < i. Scores s_j = q_t . Kbar_j (unscaled, fp32 accumulation of
+ * exact bf16 x (hi+lo bf16 split of Kbar) products). sel[b][h][t][0..k) gets
+ * the chunk ids of the top-min(k, |candidates|) candidates ordered by
+ * (score descending, chunk id ascending), padded with -1. Caption queries get
+ * all -1 (they attend densely). Q: device bf16 [B][H][L][d]; Kbar from (1);
+ * sel: device int32 [B][H][L][k]. k == 0 enqueues nothing. */
+moc_status moc_route(const moc_layout* layout, int B, int H, int d, const void* Q,
+                     const float* Kbar, int k, int causal, int32_t* sel, moc_stream_t stream);
+
+/* Bytes of device workspace moc_attention_fwd and the three stage calls need
+ * for this problem (0 on invalid arguments). Holds the per-chunk query lists,
+ * the scheduler's counters and the partial outputs (1+k fp32 rows of d plus
+ * a log-sum-exp per query). */
+size_t moc_attention_workspace_bytes(const moc_layout* layout, int B, int H, int d, int k);
+
+/* (3) Query-list builder: invert sel into per-(b, h, chunk) lists of
+ * (query, slot) entries by count -> exclusive prefix sum -> ordered scatter;
+ * each list is sorted by query index. Fills the workspace. */
+moc_status moc_build_qlists(const moc_layout* layout, int B, int H, int k, const int32_t* sel,
+                            void* ws, size_t ws_bytes, moc_stream_t stream);
+
+/* (4) Chunk-major attention over the work items (Summary §3.1 attention over
+ * Omega(q)): per 128-query tile of a query group, attention over the group's
+ * anchor key ranges (partial slot 0); per 128 entries of a chunk's query list,
+ * attention of the gathered query rows over that chunk (slot 1 + position in
+ * sel). Each partial is the normalised softmax output and its log-sum-exp of
+ * the raw scaled scores. softmax_scale is normally 1/sqrt(d). Needs the
+ * workspace filled by (3) for the same sel. */
+moc_status moc_attend_partials(const moc_layout* layout, int B, int H, int d, const void* Q,
+                               const void* K, const void* V, int k, float softmax_scale,
+                               void* ws, size_t ws_bytes, moc_stream_t stream);
+
+/* (5) Log-sum-exp merge of every query's partials: with M = max lse_j over the
+ * valid slots, w_j = exp(lse_j - M), O = sum_j w_j O_j / sum_j w_j rounded to
+ * bf16 (nearest even), lse = M + log sum_j w_j (fp32, nullable). Slots are
+ * visited in a fixed order, so the result is deterministic. */
+moc_status moc_merge(const moc_layout* layout, int B, int H, int d, int k, const int32_t* sel,
+                     void* O, float* lse, void* ws, size_t ws_bytes, moc_stream_t stream);
+
+/* Full attention stage: (3), (4) and (5) in order on one stream. */
+moc_status moc_attention_fwd(const moc_layout* layout, int B, int H, int d, const void* Q,
+                             const void* K, const void* V, const int32_t* sel, int k,
+                             float softmax_scale, void* O, float* lse, void* ws,
+                             size_t ws_bytes, moc_stream_t stream);
+
+/* Read and clear the device error word the kernels set when a bounded wait
+ * gives up or a consistency check fails. Synchronises the stream. Returns
+ * MOC_OK, MOC_ERR_DEVICE_TIMEOUT or MOC_ERR_DEVICE_CHECK; *detail (nullable)
+ * receives a kernel-specific code. */
+moc_status moc_check_device_error(void* ws, size_t ws_bytes, int32_t* detail,
+                                  moc_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOC_H */

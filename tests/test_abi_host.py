@@ -1,0 +1,130 @@
+"""C-ABI library checks that need no GPU: it loads, exports every symbol the
+header declares, builds host-only layouts whose tables agree with the oracle's
+role table, and rejects bad arguments before touching a device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import chunk_routed_sparse_b200 as moc
+import moc_workloads as W
+import oracle
+from conftest import ROOT
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "moc.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"\b(moc_[a-z_]+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = moc.lib()
+    declared = _declared_functions()
+    assert len(declared) >= 12
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(declared) == set(moc.SIGNATURES)
+
+
+def test_status_strings():
+    lib = moc.lib()
+    for s in range(8):
+        assert lib.moc_status_string(s).decode() == moc.STATUS[s]
+
+
+def _host_layout(wl):
+    return moc.Layout.from_workload(wl, device=-1)
+
+
+WORKLOADS = [W.tiny(), W.single(), W.eight(), W.ragged(), W.stress(),
+             W.tiny().replace(anchor="chunk"), W.single().replace(anchor="shot"),
+             W.ragged().replace(anchor="local", radius=2)]
+
+
+@pytest.mark.parametrize("wl", WORKLOADS, ids=lambda w: f"{w.name}-{w.anchor}")
+def test_layout_tables_agree_with_oracle_roles(wl):
+    lay = _host_layout(wl)
+    orc = oracle.Layout(wl)
+    assert lay.L == orc.L and lay.C == orc.C
+    assert lay.table(0) == orc.off.tolist()
+    grp = np.array(lay.table(1)).reshape(-1, 2)
+    ar = np.array(lay.table(2)).reshape(-1, 2)
+    ar_off = lay.table(3)
+    cand = lay.table(4)
+    cand_off = lay.table(5)
+    ncausal = lay.table(6)
+    # groups tile the token stream in order
+    assert grp[0, 0] == 0 and grp[-1, 1] == orc.L
+    assert np.all(grp[1:, 0] == grp[:-1, 1])
+    for g, (q0, q1) in enumerate(grp):
+        chunks = sorted(set(orc.chunk_of_token[q0:q1].tolist()))
+        # anchor key ranges cover exactly the tokens of the oracle's anchor chunks
+        keys = np.zeros(orc.L, dtype=bool)
+        for s, e in ar[ar_off[g]:ar_off[g + 1]]:
+            assert not keys[s:e].any()
+            keys[s:e] = True
+        for i in chunks:
+            want = (orc.role[i] == oracle.ROLE_ANCHOR)[orc.chunk_of_token]
+            assert np.array_equal(keys, want), (g, i)
+            cand_all = np.nonzero(orc.role[i] != oracle.ROLE_ANCHOR)[0]
+            cand_all = [c for c in cand_all if orc.kind[c] == W.VIDEO]
+            got = cand[cand_off[g]:cand_off[g + 1]]
+            if wl.causal:
+                assert sorted(got[:ncausal[g]]) == np.nonzero(orc.role[i] == oracle.ROLE_CAND)[0].tolist()
+            assert sorted(got) == sorted(cand_all)
+
+
+@pytest.mark.parametrize("bad", ["zero_len", "bad_kind", "split_shot", "frames_back", "anchor",
+                                 "radius", "empty"])
+def test_bad_layouts_rejected(bad):
+    ln, kind, shot, frame = [4, 5, 6, 7], [0, 1, 1, 1], [0, 0, 0, 1], [-1, 0, 1, 0]
+    anchor, radius = "shot", 0
+    if bad == "zero_len":
+        ln[2] = 0
+    elif bad == "bad_kind":
+        kind[1] = 3
+    elif bad == "split_shot":
+        shot = [0, 0, 1, 0]
+    elif bad == "frames_back":
+        frame = [-1, 1, 0, 0]
+    elif bad == "anchor":
+        anchor = 7
+    elif bad == "radius":
+        anchor, radius = "local", -1
+    elif bad == "empty":
+        ln, kind, shot, frame = [], [], [], []
+    with pytest.raises(moc.MocError) as ei:
+        moc.Layout(ln, kind, shot, frame, anchor, radius, device=-1)
+    assert ei.value.status == 2
+
+
+def test_compute_calls_reject_host_only_layout():
+    lay = _host_layout(W.tiny())
+    lib = moc.lib()
+    p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    assert lib.moc_pool_keys(lay.handle, 1, 2, 64, p, p, None) == 1
+    assert lib.moc_route(lay.handle, 1, 2, 64, p, p, 2, 1, p, None) == 1
+    assert lib.moc_attention_fwd(lay.handle, 1, 2, 64, p, p, p, p, 2, 0.125, p, None, p,
+                                 1 << 30, None) == 1
+
+
+def test_workspace_size_query():
+    wl = W.eight()
+    lay = _host_layout(wl)
+    n = lay.workspace_bytes(1, 24, 128, 3)
+    partials = 24 * wl.L * 4 * 128 * 4
+    assert partials < n < partials * 1.05
+    assert lay.workspace_bytes(1, 24, 96, 3) == 0     # d must be 64 or 128
+    assert lay.workspace_bytes(1, 24, 128, 40) == 0   # k limit
+    assert moc.lib().moc_attention_workspace_bytes(None, 1, 1, 128, 1) == 0
+
+
+def test_layout_info_counts_shots():
+    lay = _host_layout(W.ragged())
+    assert lay.n_shots == 8
+    lay1 = _host_layout(W.single())
+    assert lay1.n_shots == 1

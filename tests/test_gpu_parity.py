@@ -1,0 +1,228 @@
+"""Parity of the CUDA path (called through the C ABI) with the CPU oracle.
+
+Inputs are the seeded synthetic workloads of ``moc_workloads``; the same CPU
+bytes feed the oracle and the GPU. Tolerances are in ``tests/parity.py``.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import chunk_routed_sparse_b200 as moc
+import moc_workloads as W
+import oracle
+from parity import compare_attention, compare_routing, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    torch.cuda.init()
+
+
+def _run(wl, Q, K, V, k=None, causal=None):
+    k = wl.k if k is None else k
+    causal = wl.causal if causal is None else causal
+    lay = moc.Layout.from_workload(wl)
+    Qd, Kd, Vd = Q.cuda(), K.cuda(), V.cuda()
+    O, lse, sel, kbar = moc.forward(lay, Qd, Kd, Vd, k, causal)
+    torch.cuda.synchronize()
+    return lay, O.cpu(), lse.cpu(), sel.cpu().numpy(), kbar.cpu().numpy()
+
+
+def _check_full(wl, rows=None, k=None, n_random=0, seed=0, heads=None):
+    """Run the GPU forward on the whole problem, then check pool, routing and
+    attention of every (b, h) in ``heads`` (default: all) against the oracle,
+    on ``rows`` (None: every row; n_random > 0: boundary + random rows)."""
+    k = wl.k if k is None else k
+    wl = wl.with_k(k)
+    Q, K, V = W.make_qkv(wl, heads=heads)
+    orc = oracle.Layout(wl)
+    if rows is None and n_random:
+        rows = sample_rows(orc, n_random, seed)
+    lay, O, lse, sel, kbar = _run(wl, Q, K, V)
+    heads = heads or [(b, h) for b in range(wl.B) for h in range(wl.H)]
+    w1 = wl.replace(B=1, H=1)
+    tot = {"exact": 0, "mismatch": 0, "near": 0, "max_abs": 0.0, "mean_abs": 0.0}
+    for b, h in heads:
+        q, kk, v = (t[b:b + 1, h:h + 1].contiguous() for t in (Q, K, V))
+        kbar_o = oracle.pool(w1, kk, orc)
+        np.testing.assert_allclose(kbar[b:b + 1, h:h + 1], kbar_o, rtol=0, atol=2e-5)
+        rt = oracle.route(w1, q, kbar_o, rows=rows, lay=orc)
+        r = rt["rows"]
+        sel_g = sel[b:b + 1, h:h + 1][:, :, r, :]
+        n_eq, n_mis, n_near = compare_routing(w1, q, kbar_o, sel_g, rt, orc)
+        row_ok = np.all(rt["sel"] == sel_g, axis=-1)
+        O_o, lse_o, _ = oracle.attend(w1, q, kk, v, rt["sel"], rows=r, lay=orc)
+        mx, mean = compare_attention(O[b:b + 1, h:h + 1][:, :, r], lse[b:b + 1, h:h + 1][:, :, r],
+                                     O_o, lse_o, row_ok)
+        tot["exact"] += n_eq
+        tot["mismatch"] += n_mis
+        tot["near"] += n_near
+        tot["max_abs"] = max(tot["max_abs"], mx)
+        tot["mean_abs"] = max(tot["mean_abs"], mean)
+    return tot
+
+
+def test_tiny_all_rows():
+    res = _check_full(W.tiny())
+    assert res["mismatch"] == 0
+
+
+@pytest.mark.parametrize("k", [0, 1, 3, 8])
+def test_tiny_k_edge_cases(k):
+    """k = 0 (anchors only), k > |candidates| (shot 1 has 4): padding with -1."""
+    _check_full(W.tiny(), k=k)
+
+
+@pytest.mark.parametrize("anchor,radius,causal", [("chunk", 0, True), ("local", 1, True),
+                                                  ("shot", 0, False), ("chunk", 0, False)])
+def test_tiny_anchor_modes(anchor, radius, causal):
+    _check_full(W.tiny().replace(anchor=anchor, radius=radius, causal=causal, H=3))
+
+
+def test_small_ragged_scene_d128():
+    """Chunks shorter than a key tile, tails of every size, captions interleaved."""
+    segs = [W.Segment(37, W.CAPTION, 0, -1)]
+    lens = [1, 64, 65, 127, 128, 129, 200, 3, 300, 17]
+    for i, ln in enumerate(lens):
+        segs.append(W.Segment(ln, W.VIDEO, i // 4, i % 4))
+        if i == 3:
+            segs.append(W.Segment(5, W.CAPTION, 1, -1))
+    wl = W.custom("ragsmall", 2, 3, 128, segs, "shot", 0, True, 2, 31, "frame")
+    _check_full(wl)
+    _check_full(wl.replace(anchor="chunk"), k=5)
+
+
+def test_single_shot_clip_sampled():
+    _check_full(W.single(), n_random=512, seed=1)
+
+
+def test_eight_shot_scene_sampled():
+    """Full 180k-token eight-shot scene: routing of every row of every head,
+    attention on boundary + random rows."""
+    wl = W.eight()
+    Q, K, V = W.make_qkv(wl)
+    orc = oracle.Layout(wl)
+    lay, O, lse, sel, kbar = _run(wl, Q, K, V)
+    kbar_o = oracle.pool(wl, K, orc)
+    np.testing.assert_allclose(kbar, kbar_o, rtol=0, atol=2e-5)
+    rt = oracle.route(wl, Q, kbar_o, lay=orc)
+    n_eq, n_mis, n_near = compare_routing(wl, Q, kbar_o, sel, rt, orc)
+    print(f"eight-shot routing: exact {n_eq}, mismatched near-ties {n_mis}, near-tie rows {n_near}")
+    rows = sample_rows(orc, 256, seed=3)
+    sub = {key: (v[:, :, rows] if key in ("sel", "top_s", "top_a", "top_j", "ncand") else v)
+           for key, v in rt.items()}
+    O_o, lse_o, _ = oracle.attend(wl, Q, K, V, sub["sel"], rows=rows, lay=orc)
+    row_ok = np.all(sub["sel"] == sel[:, :, rows], axis=-1)
+    compare_attention(O[:, :, rows], lse[:, :, rows], O_o, lse_o, row_ok)
+    # pruned fraction from the GPU routing equals the oracle's count
+    kept = sum(oracle.kept_pairs(wl, sel[0, h], orc) for h in range(wl.H))
+    assert kept == wl.H * 4_943_332_144
+
+
+@pytest.mark.parametrize("k", [2, 4, 8, 16])
+def test_ragged_scene_k_sweep(k):
+    _check_full(W.ragged(), k=k, n_random=128, seed=k, heads=[(0, 0), (0, 7), (0, 23)])
+
+
+def test_stress_scene_two_heads():
+    """B=2, 361k tokens per sample, k=8: two heads carry data (the others are
+    zero and still run); checked on boundary + random rows."""
+    _check_full(W.stress(), n_random=64, seed=5, heads=[(0, 0), (1, 23)])
+
+
+def test_empty_batch_is_a_noop():
+    wl = W.tiny()
+    lay = moc.Layout.from_workload(wl)
+    Q = torch.zeros(0, 2, wl.L, 64, dtype=torch.bfloat16, device="cuda")
+    O, lse, sel, kbar = moc.forward(lay, Q, Q, Q, 2)
+    assert O.shape[0] == 0
+
+
+def test_single_chunk_scene_is_dense():
+    """One video chunk: no candidates, attention = dense over the chunk."""
+    wl = W.custom("one", 1, 2, 64, [W.Segment(300, W.VIDEO, 0, 0)], "chunk", 0, True, 3, 9, "none")
+    Q, K, V = W.make_qkv(wl)
+    lay, O, lse, sel, kbar = _run(wl, Q, K, V)
+    assert (sel == -1).all()
+    ref = torch.nn.functional.scaled_dot_product_attention(Q.double(), K.double(), V.double())
+    assert (O.double() - ref).abs().max() < 2e-2
+
+
+def test_argument_errors():
+    wl = W.tiny()
+    lay = moc.Layout.from_workload(wl)
+    Q, K, V = (t.cuda() for t in W.make_qkv(wl))
+    kbar = moc.pool_keys(lay, K)
+    sel = moc.route(lay, Q, kbar, 2)
+    ws = moc.workspace(lay, 1, 2, 64, 2)
+    O = torch.empty_like(Q)
+    lib = moc.lib()
+    s = moc._stream()
+    p = lambda t: moc._ptr(t)
+    # misaligned pointer
+    bad = torch.empty(Q.numel() * 2 + 16, dtype=torch.uint8, device="cuda")
+    assert lib.moc_pool_keys(lay.handle, 1, 2, 64, bad.data_ptr() + 2, p(kbar), s) == 1
+    # d not supported
+    assert lib.moc_pool_keys(lay.handle, 1, 2, 96, p(K), p(kbar), s) == 1
+    # k out of range
+    assert lib.moc_route(lay.handle, 1, 2, 64, p(Q), p(kbar), 32, 1, p(sel), s) == 1
+    # workspace too small
+    assert lib.moc_attention_fwd(lay.handle, 1, 2, 64, p(Q), p(K), p(V), p(sel), 2, 0.125, p(O),
+                                 None, p(ws), ws.numel() - 256, s) == 3
+    # non-positive scale
+    assert lib.moc_attention_fwd(lay.handle, 1, 2, 64, p(Q), p(K), p(V), p(sel), 2, 0.0, p(O),
+                                 None, p(ws), ws.numel(), s) == 1
+    assert moc.check_device_error(ws) == 0
+
+
+def test_qlists_invert_selection():
+    """(3) round trip: every list entry points back at its chunk; lists are
+    sorted by query and hold exactly the valid selections."""
+    wl = W.ragged(k=4, n_shots=3, H=2, d=64)
+    Q, K, V = W.make_qkv(wl)
+    lay = moc.Layout.from_workload(wl)
+    Qd, Kd, Vd = Q.cuda(), K.cuda(), V.cuda()
+    kbar = moc.pool_keys(lay, Kd)
+    sel = moc.route(lay, Qd, kbar, 4)
+    ws = moc.workspace(lay, 1, 2, 64, 4)
+    moc.build_qlists(lay, sel, 1, 2, 4, ws)
+    torch.cuda.synchronize()
+    BH, C, L, k = 2, lay.C, lay.L, 4
+    a = lambda x: (x + 255) // 256 * 256
+    nblk = (L + 1023) // 1024
+    off_qoff = a(256) + a(BH * nblk * C * 4)
+    off_tile = off_qoff + a((BH * C + 1) * 4)
+    off_list = off_tile + a((BH * C + 1) * 4)
+    wsc = ws.cpu()
+    qoff = wsc[off_qoff:off_qoff + (BH * C + 1) * 4].view(torch.int32).numpy()
+    tile = wsc[off_tile:off_tile + (BH * C + 1) * 4].view(torch.int32).numpy()
+    n_valid = int((sel >= 0).sum())
+    qlist = wsc[off_list:off_list + n_valid * 4].view(torch.int32).numpy()
+    s = sel.cpu().numpy().reshape(BH, L, k)
+    assert qoff[-1] == n_valid
+    for bh in range(BH):
+        for c in range(C):
+            x = bh * C + c
+            ent = qlist[qoff[x]:qoff[x + 1]]
+            q, slot = ent >> 5, ent & 31
+            assert np.all(np.diff(q) > 0)
+            assert np.all(s[bh, q, slot] == c)
+            want = np.nonzero((s[bh] == c).any(-1))[0]
+            assert np.array_equal(q, want)
+            assert tile[x + 1] - tile[x] == (len(ent) + 127) // 128
+
+
+def test_deterministic_repeat():
+    wl = W.tiny()
+    Q, K, V = (t.cuda() for t in W.make_qkv(wl))
+    lay = moc.Layout.from_workload(wl)
+    a = moc.forward(lay, Q, K, V, 2)
+    b = moc.forward(lay, Q, K, V, 2)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
