@@ -13,10 +13,10 @@
 //     lo = RN(x - hi)); Q is exactly bf16, so q.hi + q.lo on the tensor cores
 //     (mma.sync m16n8k16, fp32 accumulate) reproduces q.Kbar to about 2^-17
 //     relative per term instead of bf16's 2^-9;
-//   * each warp owns 16 queries and keeps their running top-k spread over its
-//     lanes (lane x holds entry x); a candidate that ranks before the current
-//     k-th entry is inserted with one ballot (its rank) and one shuffle (the
-//     shift of the worse entries). Ties rank the lower chunk id first.
+//   * the 128 x 64 scores go to shared memory and every query row is scanned
+//     by two threads (32 candidates each), each keeping a sorted top-KMAX list
+//     in registers (KMAX: compile-time bound >= k). The two lists are merged
+//     at the end. Ties rank the lower chunk id first.
 #include "common.cuh"
 
 namespace moc {
@@ -28,16 +28,32 @@ constexpr int kIdNone = 0x7fffffff;
 template <int D>
 struct RouteSmem {
     static constexpr int kStride = D + 8;  // bf16 elements per row (+16 B: conflict-free fragments)
-    static constexpr int kSStride = kCandBlock + 4;
+    static constexpr int kSStride = kCandBlock + 1;  // odd pitch: row-per-thread scans are conflict-free
     __nv_bfloat16 q[kQTile][kStride];
     __nv_bfloat16 khi[kCandBlock][kStride];
     __nv_bfloat16 klo[kCandBlock][kStride];
-    float s[8][16][kSStride];
+    float s[kQTile][kSStride];
     int cid[kCandBlock];
 };
 
-template <int D>
-__global__ void __launch_bounds__(256, 2)
+// Insert (cs, cj) into a sorted (best first) register list of KMAX entries
+// if it ranks before the last entry; the last entry drops out.
+template <int KMAX>
+__device__ __forceinline__ void topk_insert(float (&ts)[KMAX], int (&tj)[KMAX], float cs, int cj) {
+    if (!ranks_before(cs, cj, ts[KMAX - 1], tj[KMAX - 1])) return;
+    ts[KMAX - 1] = cs;
+    tj[KMAX - 1] = cj;
+#pragma unroll
+    for (int x = KMAX - 1; x > 0; --x) {
+        if (ranks_before(ts[x], tj[x], ts[x - 1], tj[x - 1])) {
+            const float fs = ts[x]; ts[x] = ts[x - 1]; ts[x - 1] = fs;
+            const int fj = tj[x]; tj[x] = tj[x - 1]; tj[x - 1] = fj;
+        }
+    }
+}
+
+template <int D, int KMAX>
+__global__ void __launch_bounds__(256, KMAX <= 16 ? 2 : 1)
     route_kernel(DevLayout dv, const __nv_bfloat16* __restrict__ Q, const float* __restrict__ Kbar,
                  int k, int causal, int32_t* __restrict__ sel) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -65,17 +81,18 @@ __global__ void __launch_bounds__(256, 2)
         if (r < nq) v = ldg_nc16(qsrc + size_t(r) * D + c * 8);
         *reinterpret_cast<uint4*>(&sm.q[r][c * 8]) = v;
     }
-    float top_s[16];
-    int top_j[16];
+    float ts[KMAX];
+    int tj[KMAX];
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
-        top_s[r] = -INFINITY;
-        top_j[r] = kIdNone;
+    for (int x = 0; x < KMAX; ++x) {
+        ts[x] = -INFINITY;
+        tj[x] = kIdNone;
     }
+    const int row = tid & (kQTile - 1), half = tid >> 7;
     const int g8 = lane >> 2, t4 = lane & 3;
     const float* kb = Kbar + size_t(bh) * dv.C * D;
     for (int cb = 0; cb < ncand; cb += kCandBlock) {
-        __syncthreads();  // previous block's candidates fully consumed
+        __syncthreads();  // previous block's candidates and scores fully consumed
         constexpr int V4 = D / 4;
         for (int i = tid; i < kCandBlock * V4; i += blockDim.x) {
             const int r = i / V4, c = i % V4;
@@ -121,73 +138,62 @@ __global__ void __launch_bounds__(256, 2)
         }
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            *reinterpret_cast<float2*>(&sm.s[warp][g8][j * 8 + 2 * t4]) = make_float2(acc[j][0], acc[j][1]);
-            *reinterpret_cast<float2*>(&sm.s[warp][g8 + 8][j * 8 + 2 * t4]) = make_float2(acc[j][2], acc[j][3]);
+            sm.s[qr + g8][j * 8 + 2 * t4] = acc[j][0];
+            sm.s[qr + g8][j * 8 + 2 * t4 + 1] = acc[j][1];
+            sm.s[qr + g8 + 8][j * 8 + 2 * t4] = acc[j][2];
+            sm.s[qr + g8 + 8][j * 8 + 2 * t4 + 1] = acc[j][3];
         }
-        __syncwarp();
+        __syncthreads();
 
-        // merge the block into each row's running top-k
-        const int j1 = sm.cid[lane], j2 = sm.cid[lane + 32];
+        // each thread scans 32 candidates of its row
+        const int nblk = min(kCandBlock, ncand - cb);
+        const int c1 = min(nblk, half * 32 + 32);
+        for (int c = half * 32; c < c1; ++c) topk_insert<KMAX>(ts, tj, sm.s[row][c], sm.cid[c]);
+    }
+    // merge the two halves of every row: half 1 publishes, half 0 merges
+    __syncthreads();
+    float* pub_s = &sm.s[0][0];
+    int* pub_j = reinterpret_cast<int*>(&sm.q[0][0]);  // q is no longer read
+    if (half == 1) {
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float s1 = (j1 == kIdNone) ? -INFINITY : sm.s[warp][r][lane];
-            float s2 = (j2 == kIdNone) ? -INFINITY : sm.s[warp][r][lane + 32];
-            float my_s = top_s[r];
-            int my_j = top_j[r];
-            float thr_s = __shfl_sync(0xffffffffu, my_s, k - 1);
-            int thr_j = __shfl_sync(0xffffffffu, my_j, k - 1);
-            unsigned m1 = __ballot_sync(0xffffffffu, ranks_before(s1, j1, thr_s, thr_j));
-            unsigned m2 = __ballot_sync(0xffffffffu, ranks_before(s2, j2, thr_s, thr_j));
-            while (m1 | m2) {
-                float cs;
-                int cj;
-                if (m1) {
-                    const int src = __ffs(m1) - 1;
-                    m1 &= m1 - 1;
-                    cs = __shfl_sync(0xffffffffu, s1, src);
-                    cj = __shfl_sync(0xffffffffu, j1, src);
-                } else {
-                    const int src = __ffs(m2) - 1;
-                    m2 &= m2 - 1;
-                    cs = __shfl_sync(0xffffffffu, s2, src);
-                    cj = __shfl_sync(0xffffffffu, j2, src);
-                }
-                if (!ranks_before(cs, cj, thr_s, thr_j)) continue;  // uniform across the warp
-                const int pos = __popc(__ballot_sync(0xffffffffu,
-                                                     lane < k && ranks_before(my_s, my_j, cs, cj)));
-                const float up_s = __shfl_up_sync(0xffffffffu, my_s, 1);
-                const int up_j = __shfl_up_sync(0xffffffffu, my_j, 1);
-                if (lane > pos) {
-                    my_s = up_s;
-                    my_j = up_j;
-                }
-                if (lane == pos) {
-                    my_s = cs;
-                    my_j = cj;
-                }
-                thr_s = __shfl_sync(0xffffffffu, my_s, k - 1);
-                thr_j = __shfl_sync(0xffffffffu, my_j, k - 1);
-            }
-            top_s[r] = my_s;
-            top_j[r] = my_j;
+        for (int x = 0; x < KMAX; ++x) {
+            pub_s[row * KMAX + x] = ts[x];
+            pub_j[row * KMAX + x] = tj[x];
         }
     }
-    const int qr = warp * 16;
+    __syncthreads();
+    if (half == 0) {
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
-        if (qr + r < nq && lane < k) out[size_t(qr + r) * k + lane] = (top_j[r] == kIdNone) ? -1 : top_j[r];
+        for (int x = 0; x < KMAX; ++x) topk_insert<KMAX>(ts, tj, pub_s[row * KMAX + x], pub_j[row * KMAX + x]);
+        if (row < nq) {
+            int32_t* o = out + size_t(row) * k;
+#pragma unroll
+            for (int x = 0; x < KMAX; ++x)
+                if (x < k) o[x] = (tj[x] == kIdNone) ? -1 : tj[x];
+        }
     }
+}
+
+template <int D, int KMAX>
+cudaError_t launch_route_dk(const DevLayout& dv, int BH, int64_t rtiles, const void* Q,
+                            const float* Kbar, int k, int causal, int32_t* sel, cudaStream_t s) {
+    const int smem = int(sizeof(RouteSmem<D>));
+    cudaError_t e = cudaFuncSetAttribute(route_kernel<D, KMAX>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(unsigned(rtiles), BH);
+    route_kernel<D, KMAX><<<grid, 256, smem, s>>>(dv, static_cast<const __nv_bfloat16*>(Q), Kbar, k,
+                                                  causal, sel);
+    return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t launch_route_d(const DevLayout& dv, int BH, int64_t rtiles, const void* Q,
                            const float* Kbar, int k, int causal, int32_t* sel, cudaStream_t s) {
-    const int smem = int(sizeof(RouteSmem<D>));
-    cudaError_t e = cudaFuncSetAttribute(route_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    dim3 grid(unsigned(rtiles), BH);
-    route_kernel<D><<<grid, 256, smem, s>>>(dv, static_cast<const __nv_bfloat16*>(Q), Kbar, k, causal, sel);
-    return cudaGetLastError();
+    if (k <= 4) return launch_route_dk<D, 4>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
+    if (k <= 8) return launch_route_dk<D, 8>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
+    if (k <= 16) return launch_route_dk<D, 16>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
+    return launch_route_dk<D, 32>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
 }
 
 }  // namespace
