@@ -1,6 +1,7 @@
 // C-ABI entry points: argument validation, workspace carve-up and kernel
 // launches. Every compute call is asynchronous on the caller's stream and
 // allocates nothing.
+#include <cstdlib>
 #include <cstring>
 
 #include "moc_internal.h"
@@ -133,8 +134,15 @@ extern "C" moc_status moc_attend_partials(const moc_layout* lay, int B, int H, i
     if (!Q || !K || !V || !aligned16(Q) || !aligned16(K) || !aligned16(V)) return MOC_ERR_INVALID_ARG;
     if (!(scale > 0.0f) || scale != scale) return MOC_ERR_INVALID_ARG;
     const int64_t n_anchor = int64_t(B) * H * lay->total_atiles;
-    return cuda_status(moc::launch_attend(lay->dv, B * H, d, Q, K, V, k, scale, n_anchor,
-                                          static_cast<char*>(ws), p, (cudaStream_t)stream));
+    static const bool use_mma = [] {
+        const char* e = getenv("MOC_ATTEND");
+        return e && strcmp(e, "mma") == 0;
+    }();
+    if (use_mma)
+        return cuda_status(moc::launch_attend_mma(lay->dv, B * H, d, Q, K, V, k, scale, n_anchor,
+                                                  static_cast<char*>(ws), p, (cudaStream_t)stream));
+    return cuda_status(moc::launch_attend_tc(lay->dv, B * H, d, Q, K, V, k, scale, n_anchor,
+                                             static_cast<char*>(ws), p, (cudaStream_t)stream));
 }
 
 extern "C" moc_status moc_merge(const moc_layout* lay, int B, int H, int d, int k,
@@ -178,7 +186,7 @@ extern "C" moc_status moc_check_device_error(void* ws, size_t ws_bytes, int32_t*
     cudaStream_t s = (cudaStream_t)stream;
     if (cudaMemcpyAsync(h, ws, sizeof h, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOC_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return MOC_ERR_CUDA;
-    if (detail) *detail = h[1];
+    if (detail) *detail = (h[0] != moc::ERR_NONE) ? h[1] : 0;
     if (h[0] != moc::ERR_NONE) {
         if (cudaMemsetAsync(ws, 0, 2 * sizeof(int32_t), s) != cudaSuccess) return MOC_ERR_CUDA;
         if (cudaStreamSynchronize(s) != cudaSuccess) return MOC_ERR_CUDA;

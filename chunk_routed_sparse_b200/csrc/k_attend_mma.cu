@@ -346,9 +346,9 @@ cudaError_t launch_d(const DevLayout& dv, int BH, const void* Q, const void* K, 
 
 }  // namespace
 
-cudaError_t launch_attend(const DevLayout& dv, int BH, int d, const void* Q, const void* K,
-                          const void* V, int k, float scale, int64_t n_anchor, char* ws,
-                          const WsPlan& p, cudaStream_t s) {
+cudaError_t launch_attend_mma(const DevLayout& dv, int BH, int d, const void* Q, const void* K,
+                              const void* V, int k, float scale, int64_t n_anchor, char* ws,
+                              const WsPlan& p, cudaStream_t s) {
     if (d == 128) return launch_d<128>(dv, BH, Q, K, V, k, scale, n_anchor, ws, p, s);
     return launch_d<64>(dv, BH, Q, K, V, k, scale, n_anchor, ws, p, s);
 }

@@ -1,0 +1,551 @@
+// (4) Chunk-major attention over work items on the 5th-generation tensor
+// cores (tcgen05 + TMEM + TMA).
+//
+// "Mixture of Contexts for Long Video Generation | Summary" §3.1: exact
+// softmax attention of q over the keys/values of Omega(q), scaled by 1/sqrt(d).
+// Omega(q) is split into disjoint parts attended separately and merged by
+// their log-sum-exp in kernel (5):
+//   anchor items - a tile of <= 128 consecutive queries of one query group
+//                  against the group's anchor key ranges (partial slot 0);
+//   routed items - <= 128 gathered queries of one chunk's query list against
+//                  that chunk's keys (slot 1 + position in sel).
+// The jxzklqfsx.com MoC write-up ("計算效率", limitations) packs these groups
+// into one variable-length FlashAttention call; here a persistent kernel
+// walks the items itself, longest first (anchor items, most keys first), then
+// routed items.
+//
+// One CTA per SM, 192 threads, warp-specialised:
+//   warp 4 (one lane): scheduler + TMA producer. Takes items from an atomic
+//          counter, publishes them in a 2-slot ring, streams 128-key K and V
+//          tiles (two 64-column, 128-byte-swizzled slabs each) into a 2-stage
+//          ring with cp.async.bulk.tensor, completion counted on mbarriers.
+//   warp 5: allocates 512 TMEM columns; one lane issues tcgen05.mma:
+//          S_j = Q K_j^T (M=128, N=128, fp32 in TMEM, double-buffered) and
+//          O += P_{j-1} V_{j-1} (M=128, N=d, V read MN-major), committing
+//          each group to the mbarrier its consumer waits on.
+//   warps 0-3: one thread per query row (= TMEM lane). Gather the item's Q
+//          rows into the swizzled shared layout, then per tile: load the S
+//          row from TMEM, mask keys past the range end, online softmax in
+//          exp2 units with a lazily updated running max (O in TMEM is only
+//          rescaled when the max grows by more than 2^8), write P as bf16 into
+//          the swizzled shared layout for the PV MMA; finally normalise O and
+//          write the partial row and its log-sum-exp.
+// Every mbarrier wait is bounded (2 s); on timeout the kernel records
+// ERR_TIMEOUT in the workspace header, every role leaves its loop, in-flight
+// copies and MMAs are drained (bounded) and TMEM is freed before exit.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace moc {
+namespace {
+
+using namespace sm100;
+
+constexpr int kKT = 128;                        // keys per tile
+constexpr int kThreads = 192;
+constexpr uint64_t kTimeoutNs = 2000000000ull;  // bounded waits
+constexpr uint32_t kTmemCols = 512;
+
+template <int D>
+struct Cfg {
+    static constexpr int kSlabs = D / 64;                // 128-byte slabs per row
+    static constexpr int kSlabBytes = 128 * 128;         // 128 rows x 128 B
+    static constexpr int kQBytes = kSlabs * kSlabBytes;  // query tile
+    static constexpr int kKVBytes = kSlabs * kSlabBytes; // one K (or V) tile
+    static constexpr int kPBytes = 2 * kSlabBytes;       // P: 128 rows x 128 keys bf16
+    static constexpr int oQ = 0;
+    static constexpr int oK = oQ + kQBytes;
+    static constexpr int oV = oK + 2 * kKVBytes;
+    static constexpr int oP = oV + 2 * kKVBytes;
+    static constexpr int oBar = oP + kPBytes;
+    // + 1024 B alignment slack; at least 120 KB so that one CTA owns an SM (and its TMEM)
+    static constexpr int kSmem = (oBar + 256 + 1024) > 120 * 1024 ? (oBar + 256 + 1024) : 120 * 1024;
+    static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, kKT, 0);
+    static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 1);
+};
+
+// mbarrier slots (8 bytes each) from Cfg::oBar
+enum {
+    B_ITEM_FULL = 0, B_ITEM_EMPTY = 2, B_KV_FULL = 4, B_KV_EMPTY = 6, B_Q_FULL = 8,
+    B_S_FULL = 9, B_S_FREE = 11, B_P_FULL = 13, B_P_FREE = 14, B_MMA_DONE = 15, B_COUNT = 16
+};
+
+struct Shared {  // at oBar + 128
+    int item[2];
+    uint32_t tmem_base;
+    int abort;
+};
+
+struct Item {
+    int bh, nq, slot_fixed, q0;
+    const int32_t* entries;
+    int r_beg, r_end, k0, k1;
+};
+
+__device__ __forceinline__ bool decode(const DevLayout& dv, int BH, int64_t n_anchor, int64_t item,
+                                       const int32_t* tile_off, const int32_t* qoff,
+                                       const int32_t* qlist, Item& it) {
+    if (item < n_anchor) {
+        const int pos = upper_index(dv.atile_off, dv.G + 1, item / BH);
+        const int64_t local = item - int64_t(BH) * dv.atile_off[pos];
+        const int nt = dv.atile_off[pos + 1] - dv.atile_off[pos];
+        const int g = dv.a_order[pos];
+        it.bh = int(local / nt);
+        it.q0 = dv.grp_q0[g] + int(local % nt) * kQTile;
+        it.nq = min(kQTile, dv.grp_q1[g] - it.q0);
+        it.slot_fixed = 0;
+        it.entries = nullptr;
+        it.r_beg = dv.ar_off[g];
+        it.r_end = dv.ar_off[g + 1];
+        it.k0 = it.k1 = 0;
+        return true;
+    }
+    const int64_t r = item - n_anchor;
+    const int64_t nlists = int64_t(BH) * dv.C;
+    if (r >= tile_off[nlists]) return false;
+    const int x = upper_index(tile_off, int(nlists + 1), r);
+    const int c = x % dv.C;
+    it.bh = x / dv.C;
+    const int e0 = qoff[x] + int(r - tile_off[x]) * kQTile;
+    it.nq = min(kQTile, qoff[x + 1] - e0);
+    it.entries = qlist + e0;
+    it.slot_fixed = -1;
+    it.q0 = 0;
+    it.r_beg = it.r_end = -1;
+    it.k0 = dv.chunk_off[c];
+    it.k1 = dv.chunk_off[c + 1];
+    return true;
+}
+
+// Key tiles of an item, in order: each range cut into 128-key tiles.
+struct Cursor {
+    const int32_t* ar;
+    int r, r_end, pos, end;
+    __device__ void init(const DevLayout& dv, const Item& it) {
+        if (it.r_beg >= 0) {
+            ar = dv.ar; r = it.r_beg; r_end = it.r_end;
+            pos = ar[2 * r];
+            end = ar[2 * r + 1];
+        } else {
+            ar = nullptr; r = 0; r_end = 1; pos = it.k0; end = it.k1;
+        }
+    }
+    __device__ bool more() const { return r < r_end; }
+    __device__ void next(int& key0, int& nvalid) {
+        key0 = pos;
+        nvalid = min(kKT, end - pos);
+        pos += kKT;
+        if (pos >= end) {
+            ++r;
+            if (ar && r < r_end) {
+                pos = ar[2 * r];
+                end = ar[2 * r + 1];
+            }
+        }
+    }
+};
+
+__device__ __forceinline__ int count_tiles(const DevLayout& dv, const Item& it) {
+    if (it.r_beg < 0) return (it.k1 - it.k0 + kKT - 1) / kKT;
+    int t = 0;
+    for (int r = it.r_beg; r < it.r_end; ++r) t += (dv.ar[2 * r + 1] - dv.ar[2 * r] + kKT - 1) / kKT;
+    return t;
+}
+
+// Bounded wait; false on timeout or when another role aborted.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort,
+                                         int32_t* hdr, int where) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63) == 0) {
+            if (*abort) return false;
+            if (globaltimer() - t0 > kTimeoutNs) {
+                set_error(hdr, ERR_TIMEOUT, where);
+                *abort = 1;
+                return false;
+            }
+        }
+    }
+}
+
+// The same wait, made uniform across the warp (the softmax warps execute
+// warp-collective tcgen05.ld/st right after it).
+__device__ __forceinline__ bool wait_bar_warp(uint32_t bar, uint32_t parity, volatile int* abort,
+                                              int32_t* hdr, int where) {
+    const bool ok = wait_bar(bar, parity, abort, hdr, where);
+    return __all_sync(0xffffffffu, ok);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attend_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                     DevLayout dv, int BH, int k, float scale_log2, int64_t n_anchor,
+                     const __nv_bfloat16* __restrict__ Q, int32_t* __restrict__ hdr,
+                     const int32_t* __restrict__ qoff, const int32_t* __restrict__ tile_off,
+                     const int32_t* __restrict__ qlist, float* __restrict__ lse_p,
+                     float* __restrict__ o_p) {
+    using C = Cfg<D>;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    // 1024-byte aligned base: the 128-byte swizzle atoms of TMA and UMMA repeat every 1024 B
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    unsigned char* gbase = smem_raw + (base - raw);
+    const uint32_t sQ = base + C::oQ, sK = base + C::oK, sV = base + C::oV, sP = base + C::oP;
+    const uint32_t sBar = base + C::oBar;
+    Shared& sh = *reinterpret_cast<Shared*>(gbase + C::oBar + 128);
+    volatile int* abort = &sh.abort;
+    auto bar = [&](int i) { return sBar + 8u * uint32_t(i); };
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int S = k + 1;
+    const size_t L = size_t(dv.L);
+
+    if (tid == 0) {
+        mbar_init(bar(B_ITEM_FULL), 1);
+        mbar_init(bar(B_ITEM_FULL + 1), 1);
+        mbar_init(bar(B_ITEM_EMPTY), 1 + 128);
+        mbar_init(bar(B_ITEM_EMPTY + 1), 1 + 128);
+        mbar_init(bar(B_KV_FULL), 1);
+        mbar_init(bar(B_KV_FULL + 1), 1);
+        mbar_init(bar(B_KV_EMPTY), 1);
+        mbar_init(bar(B_KV_EMPTY + 1), 1);
+        mbar_init(bar(B_Q_FULL), 128);
+        mbar_init(bar(B_S_FULL), 1);
+        mbar_init(bar(B_S_FULL + 1), 1);
+        mbar_init(bar(B_S_FREE), 128);
+        mbar_init(bar(B_S_FREE + 1), 128);
+        mbar_init(bar(B_P_FULL), 128);
+        mbar_init(bar(B_P_FREE), 1);
+        mbar_init(bar(B_MMA_DONE), 1);
+        sh.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(smem_u32(&sh.tmem_base), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sh.tmem_base;
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            const int64_t total = n_anchor + tile_off[int64_t(BH) * dv.C];
+            uint32_t gt = 0;
+            for (int it = 0;; ++it) {
+                const int slot = it & 1;
+                if (!wait_bar(bar(B_ITEM_EMPTY + slot), ((it >> 1) & 1) ^ 1, abort, hdr, 1)) break;
+                const int64_t item = atomicAdd(&hdr[HDR_WORK], 1);
+                const bool ok = item < total;
+                sh.item[slot] = ok ? int(item) : -1;
+                mbar_arrive(bar(B_ITEM_FULL + slot));
+                if (!ok) break;
+                Item itm;
+                decode(dv, BH, n_anchor, item, tile_off, qoff, qlist, itm);
+                Cursor cur;
+                cur.init(dv, itm);
+                const int row0 = itm.bh * dv.L;
+                bool stop = false;
+                while (cur.more()) {
+                    int key0, nvalid;
+                    cur.next(key0, nvalid);
+                    const int st = gt & 1;
+                    if (!wait_bar(bar(B_KV_EMPTY + st), ((gt >> 1) & 1) ^ 1, abort, hdr, 2)) { stop = true; break; }
+                    mbar_expect_tx(bar(B_KV_FULL + st), 2 * C::kKVBytes);
+#pragma unroll
+                    for (int s = 0; s < C::kSlabs; ++s) {
+                        tma_load_2d(sK + st * C::kKVBytes + s * C::kSlabBytes, &tmK, bar(B_KV_FULL + st), 64 * s, row0 + key0);
+                        tma_load_2d(sV + st * C::kKVBytes + s * C::kSlabBytes, &tmV, bar(B_KV_FULL + st), 64 * s, row0 + key0);
+                    }
+                    ++gt;
+                }
+                if (stop) break;
+            }
+            // drain: the last use of each stage has landed before the CTA exits
+            for (uint32_t g = (gt >= 2 ? gt - 2 : 0); g < gt; ++g) {
+                const uint32_t st = g & 1, par = (g >> 1) & 1;
+                const uint64_t t0 = globaltimer();
+                while (!mbar_try_wait(bar(B_KV_FULL + st), par)) {
+                    if (globaltimer() - t0 > kTimeoutNs) { set_error(hdr, ERR_TIMEOUT, 9); break; }
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 5) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint32_t gt = 0;
+            for (int it = 0;; ++it) {
+                const int slot = it & 1;
+                if (!wait_bar(bar(B_ITEM_FULL + slot), (it >> 1) & 1, abort, hdr, 3)) break;
+                const int item = sh.item[slot];
+                mbar_arrive(bar(B_ITEM_EMPTY + slot));
+                if (item < 0) break;
+                Item itm;
+                decode(dv, BH, n_anchor, item, tile_off, qoff, qlist, itm);
+                const int T = count_tiles(dv, itm);
+                if (!wait_bar(bar(B_Q_FULL), it & 1, abort, hdr, 4)) break;
+                tc_fence_after();
+                bool stop = false;
+                for (int j = 0; j <= T && !stop; ++j) {
+                    if (j < T) {  // S_j = Q K_j^T
+                        const uint32_t st = gt & 1, n = gt >> 1;
+                        if (!wait_bar(bar(B_KV_FULL + st), n & 1, abort, hdr, 5)) { stop = true; break; }
+                        if (!wait_bar(bar(B_S_FREE + st), (n & 1) ^ 1, abort, hdr, 6)) { stop = true; break; }
+                        tc_fence_after();
+                        const uint32_t d_s = tmem + st * kKT;
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t off = (kk >> 2) * C::kSlabBytes + (kk & 3) * 32;
+                            umma_ss(d_s, sdesc_sw128(sQ + off, 16, 1024),
+                                    sdesc_sw128(sK + st * C::kKVBytes + off, 16, 1024), C::kIdescQK,
+                                    kk > 0);
+                        }
+                        umma_commit(bar(B_S_FULL + st));
+                    }
+                    if (j > 0) {  // O += P_{j-1} V_{j-1}
+                        const uint32_t g = gt - 1, pst = g & 1;
+                        if (!wait_bar(bar(B_P_FULL), g & 1, abort, hdr, 7)) { stop = true; break; }
+                        tc_fence_after();
+                        const uint32_t d_o = tmem + 2 * kKT;
+#pragma unroll
+                        for (int kk = 0; kk < kKT / 16; ++kk) {
+                            const uint32_t aoff = (kk >> 2) * C::kSlabBytes + (kk & 3) * 32;
+                            umma_ss(d_o, sdesc_sw128(sP + aoff, 16, 1024),
+                                    sdesc_sw128(sV + pst * C::kKVBytes + kk * 2048, C::kSlabBytes, 1024),
+                                    C::kIdescPV, (j > 1 || kk > 0));
+                        }
+                        umma_commit(bar(B_P_FREE));
+                        umma_commit(bar(B_KV_EMPTY + pst));
+                    }
+                    if (j < T) ++gt;
+                }
+                if (stop) break;
+            }
+            // all issued MMAs complete before TMEM is released
+            umma_commit(bar(B_MMA_DONE));
+            const uint64_t t0 = globaltimer();
+            while (!mbar_try_wait(bar(B_MMA_DONE), 0)) {
+                if (globaltimer() - t0 > kTimeoutNs) { set_error(hdr, ERR_TIMEOUT, 10); break; }
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ softmax (warps 0-3)
+        const int row = tid;  // TMEM lane
+        const uint32_t lane_addr = tmem + (uint32_t(warp * 32) << 16);
+        uint32_t gt = 0;
+        for (int it = 0;; ++it) {
+            const int slot = it & 1;
+            if (!wait_bar_warp(bar(B_ITEM_FULL + slot), (it >> 1) & 1, abort, hdr, 11)) break;
+            const int item = sh.item[slot];
+            mbar_arrive(bar(B_ITEM_EMPTY + slot));
+            if (item < 0) break;
+            Item itm;
+            decode(dv, BH, n_anchor, item, tile_off, qoff, qlist, itm);
+            const __nv_bfloat16* Qb = Q + size_t(itm.bh) * L * D;
+            // this thread's row: token and partial slot
+            int my_tok = -1, my_slot = 0;
+            if (row < itm.nq) {
+                if (itm.slot_fixed >= 0) {
+                    my_tok = itm.q0 + row;
+                } else {
+                    const int e = itm.entries[row];
+                    my_tok = e >> 5;
+                    my_slot = 1 + (e & 31);
+                }
+            }
+            // gather the warp's 32 query rows (2 rows x 16 B chunks per step)
+            constexpr int CH = D / 8;  // 16-byte chunks per row
+#pragma unroll 4
+            for (int i = 0; i < 32 * CH / 32; ++i) {
+                const int idx = i * 32 + lane;
+                const int r = warp * 32 + idx / CH, ch = idx % CH;
+                const int tok = __shfl_sync(0xffffffffu, my_tok, r & 31);
+                uint4 v = make_uint4(0, 0, 0, 0);
+                if (tok >= 0) v = ldg_nc16(Qb + size_t(tok) * D + ch * 8);
+                const uint32_t dst = sQ + (ch >> 3) * C::kSlabBytes + r * 128 + (((ch & 7) ^ (r & 7)) << 4);
+                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(v.x), "r"(v.y),
+                             "r"(v.z), "r"(v.w) : "memory");
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(bar(B_Q_FULL));
+
+            Cursor cur;
+            cur.init(dv, itm);
+            float m_used = -INFINITY, l = 0.f;
+            bool stop = false;
+            for (int j = 0; cur.more(); ++j) {
+                int key0, nvalid;
+                cur.next(key0, nvalid);
+                const uint32_t sb = gt & 1, n = gt >> 1;
+                if (!wait_bar_warp(bar(B_S_FULL + sb), n & 1, abort, hdr, 12)) { stop = true; break; }
+                tc_fence_after();
+                uint32_t s[kKT];
+#pragma unroll
+                for (int c = 0; c < kKT / 32; ++c)
+                    tmem_ld32(lane_addr + sb * kKT + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(bar(B_S_FREE + sb));
+                // scale (log2 units), mask keys past the range end, row max
+                float mx = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < kKT; ++c) {
+                    const float v = (c < nvalid) ? __uint_as_float(s[c]) * scale_log2 : -INFINITY;
+                    s[c] = __float_as_uint(v);
+                    mx = fmaxf(mx, v);
+                }
+                float alpha = 1.f;
+                bool rescale = false;
+                if (j == 0) {
+                    m_used = mx;
+                } else if (mx > m_used + 8.f) {  // lazy rescale: only when the max grew by > 2^8
+                    alpha = ex2(m_used - mx);
+                    m_used = mx;
+                    rescale = true;
+                }
+                float rs = 0.f;
+                uint32_t pk[kKT / 2];
+#pragma unroll
+                for (int c = 0; c < kKT; c += 2) {
+                    const float p0 = ex2(__uint_as_float(s[c]) - m_used);
+                    const float p1 = ex2(__uint_as_float(s[c + 1]) - m_used);
+                    rs += p0 + p1;
+                    pk[c / 2] = pack_bf16(p0, p1);
+                }
+                l = l * alpha + rs;
+                if (j > 0) {  // PV of the previous tile done: P buffer free, O current
+                    if (!wait_bar_warp(bar(B_P_FREE), (gt - 1) & 1, abort, hdr, 13)) { stop = true; break; }
+                    tc_fence_after();
+                }
+                if (__any_sync(0xffffffffu, rescale)) {  // warp-collective TMEM access; alpha = 1 elsewhere
+                    const uint32_t o_addr = lane_addr + 2 * kKT;
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(o_addr + c * 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+                        tmem_st32(o_addr + c * 32, o);
+                    }
+                    tmem_wait_st();
+                }
+                // P row -> shared memory, 128-byte swizzle (16 chunks of 8 keys)
+#pragma unroll
+                for (int ch = 0; ch < kKT / 8; ++ch) {
+                    const uint32_t dst = sP + (ch >> 3) * C::kSlabBytes + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
+                    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(pk[ch * 4]),
+                                 "r"(pk[ch * 4 + 1]), "r"(pk[ch * 4 + 2]), "r"(pk[ch * 4 + 3]) : "memory");
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(bar(B_P_FULL));
+                ++gt;
+            }
+            if (stop) break;
+            // epilogue: final PV done -> O / l -> partial row, log-sum-exp
+            if (!wait_bar_warp(bar(B_P_FREE), (gt - 1) & 1, abort, hdr, 14)) break;
+            tc_fence_after();
+            const float inv = 1.f / l;
+            const uint32_t o_addr = lane_addr + 2 * kKT;
+            float* dst = (my_tok >= 0) ? o_p + ((size_t(itm.bh) * L + my_tok) * S + my_slot) * D : nullptr;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(o_addr + c * 32, o);
+                tmem_wait_ld();
+                if (dst) {
+#pragma unroll
+                    for (int x = 0; x < 32; x += 4) {
+                        float4 v = make_float4(__uint_as_float(o[x]) * inv, __uint_as_float(o[x + 1]) * inv,
+                                               __uint_as_float(o[x + 2]) * inv, __uint_as_float(o[x + 3]) * inv);
+                        *reinterpret_cast<float4*>(dst + c * 32 + x) = v;
+                    }
+                }
+            }
+            tc_fence_before();
+            if (dst) lse_p[(size_t(itm.bh) * L + my_tok) * S + my_slot] = (m_used + log2f(l)) * 0.69314718055994531f;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// [rows][d] bf16 matrix, box = 64 columns (128 B) x 128 rows, 128-byte swizzle
+bool make_tmap(CUtensorMap* tm, const void* ptr, int d, int64_t rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(rows)};
+    cuuint64_t strides[1] = {cuuint64_t(d) * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch_d(const DevLayout& dv, int BH, const void* Q, const void* K, const void* V, int k,
+                     float scale, int64_t n_anchor, char* ws, const WsPlan& p, cudaStream_t s) {
+    CUtensorMap tmK, tmV;
+    const int64_t rows = int64_t(BH) * dv.L;
+    if (!make_tmap(&tmK, K, D, rows) || !make_tmap(&tmV, V, D, rows)) return cudaErrorInvalidValue;
+    const int smem = Cfg<D>::kSmem;
+    cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int32_t* hdr = reinterpret_cast<int32_t*>(ws + p.hdr);
+    e = cudaMemsetAsync(hdr + HDR_WORK, 0, sizeof(int32_t), s);
+    if (e != cudaSuccess) return e;
+    attend_tc_kernel<D><<<sms, kThreads, smem, s>>>(
+        tmK, tmV, dv, BH, k, scale * 1.4426950408889634f, n_anchor, static_cast<const __nv_bfloat16*>(Q), hdr,
+        reinterpret_cast<const int32_t*>(ws + p.qoff), reinterpret_cast<const int32_t*>(ws + p.tile_off),
+        reinterpret_cast<const int32_t*>(ws + p.qlist), reinterpret_cast<float*>(ws + p.lse_p),
+        reinterpret_cast<float*>(ws + p.o_p));
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attend_tc(const DevLayout& dv, int BH, int d, const void* Q, const void* K,
+                             const void* V, int k, float scale, int64_t n_anchor, char* ws,
+                             const WsPlan& p, cudaStream_t s) {
+    if (d == 128) return launch_d<128>(dv, BH, Q, K, V, k, scale, n_anchor, ws, p, s);
+    return launch_d<64>(dv, BH, Q, K, V, k, scale, n_anchor, ws, p, s);
+}
+
+}  // namespace moc

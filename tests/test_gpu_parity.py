@@ -178,6 +178,8 @@ def test_argument_errors():
     # non-positive scale
     assert lib.moc_attention_fwd(lay.handle, 1, 2, 64, p(Q), p(K), p(V), p(sel), 2, 0.0, p(O),
                                  None, p(ws), ws.numel(), s) == 1
+    # a good call after the rejected ones: it clears and leaves a clean device error word
+    moc.attention_fwd(lay, Q, K, V, sel, 2, ws=ws, O=O)
     assert moc.check_device_error(ws) == 0
 
 
