@@ -65,6 +65,7 @@ SIGNATURES = {
     "moc_attend_partials": (_I, [_P, _I, _I, _I, _P, _P, _P, _I, _F, _P, _SZ, _P]),
     "moc_merge": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _SZ, _P]),
     "moc_attention_fwd": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _F, _P, _P, _P, _SZ, _P]),
+    "moc_attention_fwd_static": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _F, _P, _P, _P]),
     "moc_check_device_error": (_I, [_P, _SZ, _P, _P]),
 }
 

@@ -170,6 +170,22 @@ moc_status moc_attention_fwd(const moc_layout* layout, int B, int H, int d, cons
                              float softmax_scale, void* O, float* lse, void* ws,
                              size_t ws_bytes, moc_stream_t stream);
 
+/* moc_attention_fwd without a caller workspace, for callers that cannot
+ * allocate device memory (a plugin given only its input and output buffers, a
+ * real-time loop that must stay off the driver's allocation path, code running
+ * while a framework's allocator is frozen for graph capture). The pages
+ * describe no counterpart: this is a deployment variant of (3)-(5) above.
+ * Scratch: a static 64 MiB device array inside the library, held on every GPU
+ * that loads it until the process exits; nothing is allocated per call.
+ * Returns MOC_ERR_WORKSPACE_TOO_SMALL when moc_attention_workspace_bytes()
+ * for the problem exceeds 64 MiB. The first call on a device looks up the
+ * array's device address (make that first call before any stream capture).
+ * All calls share the array: calls that overlap on the GPU race. Arguments
+ * otherwise as moc_attention_fwd. */
+moc_status moc_attention_fwd_static(const moc_layout* layout, int B, int H, int d, const void* Q,
+                                    const void* K, const void* V, const int32_t* sel, int k,
+                                    float softmax_scale, void* O, float* lse, moc_stream_t stream);
+
 /* Read and clear the device error word the kernels set when a bounded wait
  * gives up or a consistency check fails. Synchronises the stream. Returns
  * MOC_OK, MOC_ERR_DEVICE_TIMEOUT or MOC_ERR_DEVICE_CHECK; *detail (nullable)
