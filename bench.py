@@ -120,8 +120,6 @@ def kernel_traffic():
     """Per-launch DRAM bytes of the attend kernel from the committed ncu
     summary, if it was taken on the current kernel source (else None)."""
     src = os.path.join(ROOT, "chunk_routed_sparse_b200", "csrc", "k_attend_tc.cu")
-    if not os.path.exists(src):
-        src = os.path.join(ROOT, "chunk_routed_sparse_b200", "csrc", "k_attend_mma.cu")
     summ = os.path.join(ROOT, "profiles", "attend_traffic.txt")
     if not os.path.exists(summ):
         return None
@@ -152,6 +150,21 @@ def selected_pairs(layout_tables, wl, sel: torch.Tensor) -> int:
     return anchor + routed
 
 
+def scene_for_rank(wl, rank: int):
+    """Weak scaling: every rank runs an independent scene of the same shape."""
+    return wl.replace(seed=wl.seed + 1000 * rank)
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over all ranks (identity at N=1)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
 def run_ours(args):
     import chunk_routed_sparse_b200 as moc
 
@@ -162,8 +175,7 @@ def run_ours(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    wl = workload(args.config, args.k)
-    wl = wl.replace(seed=wl.seed + 1000 * rank)  # an independent scene per rank
+    wl = scene_for_rank(workload(args.config, args.k), rank)
     B, H, L, d, k = wl.B, wl.H, wl.L, wl.d, wl.k
     Qh, Kh, Vh = W.make_qkv(wl)
     Qh, Kh, Vh = Qh.pin_memory(), Kh.pin_memory(), Vh.pin_memory()
@@ -240,10 +252,7 @@ def run_ours(args):
     barrier()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
 
-    if ws_ > 1:
-        t = torch.tensor([total_ms, e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms, e2e_ms = float(t[0]), float(t[1])
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
 
     ms_per_step = total_ms / args.steps
     tokens = B * L

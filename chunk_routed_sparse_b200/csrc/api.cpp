@@ -1,7 +1,6 @@
 // C-ABI entry points: argument validation, workspace carve-up and kernel
 // launches. Every compute call is asynchronous on the caller's stream and
 // allocates nothing.
-#include <cstdlib>
 #include <cstring>
 
 #include "moc_internal.h"
@@ -134,13 +133,6 @@ extern "C" moc_status moc_attend_partials(const moc_layout* lay, int B, int H, i
     if (!Q || !K || !V || !aligned16(Q) || !aligned16(K) || !aligned16(V)) return MOC_ERR_INVALID_ARG;
     if (!(scale > 0.0f) || scale != scale) return MOC_ERR_INVALID_ARG;
     const int64_t n_anchor = int64_t(B) * H * lay->total_atiles;
-    static const bool use_mma = [] {
-        const char* e = getenv("MOC_ATTEND");
-        return e && strcmp(e, "mma") == 0;
-    }();
-    if (use_mma)
-        return cuda_status(moc::launch_attend_mma(lay->dv, B * H, d, Q, K, V, k, scale, n_anchor,
-                                                  static_cast<char*>(ws), p, (cudaStream_t)stream));
     return cuda_status(moc::launch_attend_tc(lay->dv, B * H, d, Q, K, V, k, scale, n_anchor,
                                              static_cast<char*>(ws), p, (cudaStream_t)stream));
 }

@@ -78,9 +78,6 @@ cudaError_t launch_qlists(const DevLayout& dv, int BH, int k, const int32_t* sel
 cudaError_t launch_attend_tc(const DevLayout& dv, int BH, int d, const void* Q, const void* K,
                              const void* V, int k, float scale, int64_t n_anchor_items, char* ws,
                              const WsPlan& p, cudaStream_t s);
-cudaError_t launch_attend_mma(const DevLayout& dv, int BH, int d, const void* Q, const void* K,
-                              const void* V, int k, float scale, int64_t n_anchor_items, char* ws,
-                              const WsPlan& p, cudaStream_t s);
 cudaError_t launch_merge(int BH, int L, int d, int k, const int32_t* sel, void* O, float* lse,
                          const char* ws, const WsPlan& p, cudaStream_t s);
 
