@@ -5,34 +5,40 @@
 // softmax attention of q over the keys/values of Omega(q), scaled by 1/sqrt(d).
 // Omega(q) is split into disjoint parts attended separately and merged by
 // their log-sum-exp in kernel (5):
-//   anchor items - a tile of <= 128 consecutive queries of one query group
-//                  against the group's anchor key ranges (partial slot 0);
-//   routed items - <= 128 gathered queries of one chunk's query list against
+//   anchor items - <= 256 consecutive queries of one query group against the
+//                  group's anchor key ranges (partial slot 0);
+//   routed items - <= 256 gathered queries of one chunk's query list against
 //                  that chunk's keys (slot 1 + position in sel).
 // The jxzklqfsx.com MoC write-up ("計算效率", limitations) packs these groups
-// into one variable-length FlashAttention call; here a persistent kernel
-// walks the items itself, longest first (anchor items, most keys first), then
-// routed items.
+// into one variable-length FlashAttention call; here a persistent kernel walks
+// the items itself, longest first (anchor items, most keys first), then routed
+// items.
 //
-// One CTA per SM, 192 threads, warp-specialised:
-//   warp 4 (one lane): scheduler + TMA producer. Takes items from an atomic
+// One CTA per SM, 384 threads, warp-specialised. An item's rows form two
+// 128-row tiles A and B that share one K/V stream:
+//   warp 8 (one lane): scheduler + TMA producer. Takes items from an atomic
 //          counter, publishes them in a 2-slot ring, streams 128-key K and V
-//          tiles (two 64-column, 128-byte-swizzled slabs each) into a 2-stage
-//          ring with cp.async.bulk.tensor, completion counted on mbarriers.
-//   warp 5: allocates 512 TMEM columns; one lane issues tcgen05.mma:
-//          S_j = Q K_j^T (M=128, N=128, fp32 in TMEM, double-buffered) and
-//          O += P_{j-1} V_{j-1} (M=128, N=d, V read MN-major), committing
-//          each group to the mbarrier its consumer waits on.
-//   warps 0-3: one thread per query row (= TMEM lane). Gather the item's Q
-//          rows into the swizzled shared layout, then per tile: load the S
-//          row from TMEM, mask keys past the range end, online softmax in
-//          exp2 units with a lazily updated running max (O in TMEM is only
-//          rescaled when the max grows by more than 2^8), write P as bf16 into
-//          the swizzled shared layout for the PV MMA; finally normalise O and
-//          write the partial row and its log-sum-exp.
-// Every mbarrier wait is bounded (2 s); on timeout the kernel records
-// ERR_TIMEOUT in the workspace header, every role leaves its loop, in-flight
-// copies and MMAs are drained (bounded) and TMEM is freed before exit.
+//          tiles (64-column, 128-byte-swizzled slabs) into a 2-stage ring with
+//          cp.async.bulk.tensor, completion counted on mbarriers.
+//          (warps 10-11 only complete the third warpgroup.)
+//   warp 9: allocates all 512 TMEM columns (S_A, S_B, O_A, O_B); one lane
+//          issues tcgen05.mma in the order
+//            S_A(0) S_B(0) | PV_A(0) S_A(1) PV_B(0) S_B(1) | PV_A(1) S_A(2) ...
+//          with S = Q K^T (M=128, N=128, fp32 in TMEM) and O += P V where P is
+//          read from TMEM (bf16, written over its own S columns) and V from
+//          shared memory (MN-major). While the tensor core works on one tile's
+//          PV and next S, the other tile's softmax runs (ping-pong).
+//   warps 0-3 / 4-7: softmax of tile A / tile B, one thread per query row
+//          (= TMEM lane). Gather the tile's Q rows into the swizzled shared
+//          layout; per key tile: load the S row from TMEM, mask keys past the
+//          range end, online softmax in exp2 units with a lazily updated
+//          running max (O is only rescaled in TMEM when the max grows by more
+//          than 2^8, exact because the final normalisation uses the same max),
+//          store P as bf16 back into TMEM; finally normalise O and write the
+//          partial row and its log-sum-exp.
+// Every mbarrier wait is bounded (2 s): on timeout the kernel records
+// ERR_TIMEOUT and a site code in the workspace header, every role leaves its
+// loop, in-flight copies and MMAs are drained (bounded) and TMEM is freed.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -44,35 +50,42 @@ namespace {
 using namespace sm100;
 
 constexpr int kKT = 128;                        // keys per tile
-constexpr int kThreads = 192;
+constexpr int kThreads = 384;                   // softmax A, softmax B, producer/MMA warpgroups
+// Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64512);
+// the producer/MMA warpgroup drops to 72 and the softmax warpgroups rise to
+// 216: 2 x 128 x 216 + 128 x 72 = 64512, and per SM sub-partition
+// (one warp of each warpgroup) 32 x (216 + 216 + 72) = 16128 <= 16384.
+constexpr int kRegsSoftmax = 216;
+constexpr int kRegsOther = 72;
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // bounded waits
 constexpr uint32_t kTmemCols = 512;
 
 template <int D>
 struct Cfg {
-    static constexpr int kSlabs = D / 64;                // 128-byte slabs per row
-    static constexpr int kSlabBytes = 128 * 128;         // 128 rows x 128 B
-    static constexpr int kQBytes = kSlabs * kSlabBytes;  // query tile
-    static constexpr int kKVBytes = kSlabs * kSlabBytes; // one K (or V) tile
-    static constexpr int kPBytes = 2 * kSlabBytes;       // P: 128 rows x 128 keys bf16
-    static constexpr int oQ = 0;
-    static constexpr int oK = oQ + kQBytes;
-    static constexpr int oV = oK + 2 * kKVBytes;
-    static constexpr int oP = oV + 2 * kKVBytes;
-    static constexpr int oBar = oP + kPBytes;
+    static constexpr int kSlabs = D / 64;                   // 128-byte slabs per row
+    static constexpr int kSlabBytes = 128 * 128;            // 128 rows x 128 B
+    static constexpr int kTileBytes = kSlabs * kSlabBytes;  // a 128-row Q, K or V tile
+    static constexpr int oQ = 0;                            // Q_A, Q_B
+    static constexpr int oK = oQ + 2 * kTileBytes;          // 2 stages
+    static constexpr int oV = oK + 2 * kTileBytes;          // 2 stages
+    static constexpr int oBar = oV + 2 * kTileBytes;
     // + 1024 B alignment slack; at least 120 KB so that one CTA owns an SM (and its TMEM)
     static constexpr int kSmem = (oBar + 256 + 1024) > 120 * 1024 ? (oBar + 256 + 1024) : 120 * 1024;
     static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, kKT, 0);
     static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 1);
 };
 
-// mbarrier slots (8 bytes each) from Cfg::oBar
+// TMEM columns: S_A / S_B (P_A / P_B overwrite their first 64 columns), O_A / O_B
+__device__ __forceinline__ uint32_t col_s(int q) { return q ? 128u : 0u; }
+__device__ __forceinline__ uint32_t col_o(int q) { return q ? 384u : 256u; }
+
+// mbarrier slots (8 bytes each) from Cfg::oBar; [x] = tile A / B or ring slot
 enum {
     B_ITEM_FULL = 0, B_ITEM_EMPTY = 2, B_KV_FULL = 4, B_KV_EMPTY = 6, B_Q_FULL = 8,
-    B_S_FULL = 9, B_S_FREE = 11, B_P_FULL = 13, B_P_FREE = 14, B_MMA_DONE = 15, B_COUNT = 16
+    B_S_FULL = 10, B_P_FULL = 12, B_PV_DONE = 14, B_MMA_DONE = 16, B_COUNT = 17
 };
 
-struct Shared {  // at oBar + 128
+struct Shared {  // at oBar + 192
     int item[2];
     uint32_t tmem_base;
     int abort;
@@ -93,8 +106,8 @@ __device__ __forceinline__ bool decode(const DevLayout& dv, int BH, int64_t n_an
         const int nt = dv.atile_off[pos + 1] - dv.atile_off[pos];
         const int g = dv.a_order[pos];
         it.bh = int(local / nt);
-        it.q0 = dv.grp_q0[g] + int(local % nt) * kQTile;
-        it.nq = min(kQTile, dv.grp_q1[g] - it.q0);
+        it.q0 = dv.grp_q0[g] + int(local % nt) * kItemRows;
+        it.nq = min(kItemRows, dv.grp_q1[g] - it.q0);
         it.slot_fixed = 0;
         it.entries = nullptr;
         it.r_beg = dv.ar_off[g];
@@ -108,8 +121,8 @@ __device__ __forceinline__ bool decode(const DevLayout& dv, int BH, int64_t n_an
     const int x = upper_index(tile_off, int(nlists + 1), r);
     const int c = x % dv.C;
     it.bh = x / dv.C;
-    const int e0 = qoff[x] + int(r - tile_off[x]) * kQTile;
-    it.nq = min(kQTile, qoff[x + 1] - e0);
+    const int e0 = qoff[x] + int(r - tile_off[x]) * kItemRows;
+    it.nq = min(kItemRows, qoff[x + 1] - e0);
     it.entries = qlist + e0;
     it.slot_fixed = -1;
     it.q0 = 0;
@@ -194,9 +207,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     unsigned char* gbase = smem_raw + (base - raw);
-    const uint32_t sQ = base + C::oQ, sK = base + C::oK, sV = base + C::oV, sP = base + C::oP;
+    const uint32_t sQ = base + C::oQ, sK = base + C::oK, sV = base + C::oV;
     const uint32_t sBar = base + C::oBar;
-    Shared& sh = *reinterpret_cast<Shared*>(gbase + C::oBar + 128);
+    Shared& sh = *reinterpret_cast<Shared*>(gbase + C::oBar + 192);
     volatile int* abort = &sh.abort;
     auto bar = [&](int i) { return sBar + 8u * uint32_t(i); };
 
@@ -205,26 +218,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     const size_t L = size_t(dv.L);
 
     if (tid == 0) {
-        mbar_init(bar(B_ITEM_FULL), 1);
-        mbar_init(bar(B_ITEM_FULL + 1), 1);
-        mbar_init(bar(B_ITEM_EMPTY), 1 + 128);
-        mbar_init(bar(B_ITEM_EMPTY + 1), 1 + 128);
-        mbar_init(bar(B_KV_FULL), 1);
-        mbar_init(bar(B_KV_FULL + 1), 1);
-        mbar_init(bar(B_KV_EMPTY), 1);
-        mbar_init(bar(B_KV_EMPTY + 1), 1);
-        mbar_init(bar(B_Q_FULL), 128);
-        mbar_init(bar(B_S_FULL), 1);
-        mbar_init(bar(B_S_FULL + 1), 1);
-        mbar_init(bar(B_S_FREE), 128);
-        mbar_init(bar(B_S_FREE + 1), 128);
-        mbar_init(bar(B_P_FULL), 128);
-        mbar_init(bar(B_P_FREE), 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(bar(B_ITEM_FULL + x), 1);
+            mbar_init(bar(B_ITEM_EMPTY + x), 1 + 256);
+            mbar_init(bar(B_KV_FULL + x), 1);
+            mbar_init(bar(B_KV_EMPTY + x), 1);
+            mbar_init(bar(B_Q_FULL + x), 128);
+            mbar_init(bar(B_S_FULL + x), 1);
+            mbar_init(bar(B_P_FULL + x), 128);
+            mbar_init(bar(B_PV_DONE + x), 1);
+        }
         mbar_init(bar(B_MMA_DONE), 1);
         sh.abort = 0;
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == 9) {
         tmem_alloc(smem_u32(&sh.tmem_base), kTmemCols);
         tmem_relinquish();
     }
@@ -233,7 +241,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = sh.tmem_base;
 
-    if (warp == 4) {
+    if (warp >= 8) {
+      regs_dec<kRegsOther>();
+      if (warp == 8) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tmap(&tmK);
@@ -259,11 +269,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     cur.next(key0, nvalid);
                     const int st = gt & 1;
                     if (!wait_bar(bar(B_KV_EMPTY + st), ((gt >> 1) & 1) ^ 1, abort, hdr, 2)) { stop = true; break; }
-                    mbar_expect_tx(bar(B_KV_FULL + st), 2 * C::kKVBytes);
+                    mbar_expect_tx(bar(B_KV_FULL + st), 2 * C::kTileBytes);
 #pragma unroll
                     for (int s = 0; s < C::kSlabs; ++s) {
-                        tma_load_2d(sK + st * C::kKVBytes + s * C::kSlabBytes, &tmK, bar(B_KV_FULL + st), 64 * s, row0 + key0);
-                        tma_load_2d(sV + st * C::kKVBytes + s * C::kSlabBytes, &tmV, bar(B_KV_FULL + st), 64 * s, row0 + key0);
+                        tma_load_2d(sK + st * C::kTileBytes + s * C::kSlabBytes, &tmK, bar(B_KV_FULL + st), 64 * s, row0 + key0);
+                        tma_load_2d(sV + st * C::kTileBytes + s * C::kSlabBytes, &tmV, bar(B_KV_FULL + st), 64 * s, row0 + key0);
                     }
                     ++gt;
                 }
@@ -279,11 +289,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         __syncwarp();
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            uint32_t gt = 0;
-            for (int it = 0;; ++it) {
+            uint32_t gt = 0;           // key tiles of all items (K/V ring)
+            uint32_t gtt[2] = {0, 0};  // key tiles per query tile (S_FULL / P_FULL / PV_DONE phases)
+            uint32_t itq[2] = {0, 0};  // items per query tile (Q_FULL phases)
+            bool stop = false;
+            for (int it = 0; !stop; ++it) {
                 const int slot = it & 1;
                 if (!wait_bar(bar(B_ITEM_FULL + slot), (it >> 1) & 1, abort, hdr, 3)) break;
                 const int item = sh.item[slot];
@@ -292,43 +305,48 @@ __global__ void __launch_bounds__(kThreads, 1)
                 Item itm;
                 decode(dv, BH, n_anchor, item, tile_off, qoff, qlist, itm);
                 const int T = count_tiles(dv, itm);
-                if (!wait_bar(bar(B_Q_FULL), it & 1, abort, hdr, 4)) break;
+                const int nt = itm.nq > kQTile ? 2 : 1;  // query tiles in this item
+                for (int q = 0; q < nt && !stop; ++q)
+                    if (!wait_bar(bar(B_Q_FULL + q), itq[q] & 1, abort, hdr, 4)) stop = true;
+                if (stop) break;
                 tc_fence_after();
-                bool stop = false;
                 for (int j = 0; j <= T && !stop; ++j) {
-                    if (j < T) {  // S_j = Q K_j^T
-                        const uint32_t st = gt & 1, n = gt >> 1;
-                        if (!wait_bar(bar(B_KV_FULL + st), n & 1, abort, hdr, 5)) { stop = true; break; }
-                        if (!wait_bar(bar(B_S_FREE + st), (n & 1) ^ 1, abort, hdr, 6)) { stop = true; break; }
-                        tc_fence_after();
-                        const uint32_t d_s = tmem + st * kKT;
+                    const uint32_t st = gt & 1;
+                    bool kv_ready = false;
+                    for (int q = 0; q < nt; ++q) {
+                        if (j > 0) {  // O_q += P_q(j-1) V(j-1)
+                            const uint32_t g = gtt[q] - 1, pst = (gt - 1) & 1;
+                            if (!wait_bar(bar(B_P_FULL + q), g & 1, abort, hdr, 7)) { stop = true; break; }
+                            tc_fence_after();
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t off = (kk >> 2) * C::kSlabBytes + (kk & 3) * 32;
-                            umma_ss(d_s, sdesc_sw128(sQ + off, 16, 1024),
-                                    sdesc_sw128(sK + st * C::kKVBytes + off, 16, 1024), C::kIdescQK,
-                                    kk > 0);
+                            for (int kk = 0; kk < kKT / 16; ++kk)
+                                umma_ts(tmem + col_o(q), tmem + col_s(q) + kk * 8,
+                                        sdesc_sw128(sV + pst * C::kTileBytes + kk * 2048, C::kSlabBytes, 1024),
+                                        C::kIdescPV, (j > 1 || kk > 0));
+                            umma_commit(bar(B_PV_DONE + q));
                         }
-                        umma_commit(bar(B_S_FULL + st));
-                    }
-                    if (j > 0) {  // O += P_{j-1} V_{j-1}
-                        const uint32_t g = gt - 1, pst = g & 1;
-                        if (!wait_bar(bar(B_P_FULL), g & 1, abort, hdr, 7)) { stop = true; break; }
-                        tc_fence_after();
-                        const uint32_t d_o = tmem + 2 * kKT;
+                        if (j < T) {  // S_q(j) = Q_q K(j)^T, after PV_q(j-1) has read P_q(j-1)
+                            if (!kv_ready) {
+                                if (!wait_bar(bar(B_KV_FULL + st), (gt >> 1) & 1, abort, hdr, 5)) { stop = true; break; }
+                                kv_ready = true;
+                                tc_fence_after();
+                            }
+                            const uint32_t qb = sQ + q * C::kTileBytes, kb = sK + st * C::kTileBytes;
 #pragma unroll
-                        for (int kk = 0; kk < kKT / 16; ++kk) {
-                            const uint32_t aoff = (kk >> 2) * C::kSlabBytes + (kk & 3) * 32;
-                            umma_ss(d_o, sdesc_sw128(sP + aoff, 16, 1024),
-                                    sdesc_sw128(sV + pst * C::kKVBytes + kk * 2048, C::kSlabBytes, 1024),
-                                    C::kIdescPV, (j > 1 || kk > 0));
+                            for (int kk = 0; kk < D / 16; ++kk) {
+                                const uint32_t off = (kk >> 2) * C::kSlabBytes + (kk & 3) * 32;
+                                umma_ss(tmem + col_s(q), sdesc_sw128(qb + off, 16, 1024),
+                                        sdesc_sw128(kb + off, 16, 1024), C::kIdescQK, kk > 0);
+                            }
+                            umma_commit(bar(B_S_FULL + q));
+                            ++gtt[q];
                         }
-                        umma_commit(bar(B_P_FREE));
-                        umma_commit(bar(B_KV_EMPTY + pst));
                     }
+                    if (stop) break;
+                    if (j > 0) umma_commit(bar(B_KV_EMPTY + ((gt - 1) & 1)));  // K(j-1), V(j-1) read
                     if (j < T) ++gt;
                 }
-                if (stop) break;
+                for (int q = 0; q < nt; ++q) ++itq[q];
             }
             // all issued MMAs complete before TMEM is released
             umma_commit(bar(B_MMA_DONE));
@@ -338,11 +356,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         __syncwarp();
+    }
     } else {
-        // ------------------------------------------------------------ softmax (warps 0-3)
-        const int row = tid;  // TMEM lane
-        const uint32_t lane_addr = tmem + (uint32_t(warp * 32) << 16);
-        uint32_t gt = 0;
+        regs_inc<kRegsSoftmax>();
+        // ------------------------------------------------------------ softmax (warps 0-7)
+        const int q = warp >> 2;    // query tile A (0) or B (1)
+        const int row = tid & 127;  // row within the tile = TMEM lane
+        const uint32_t lane_addr = tmem + (uint32_t((warp & 3) * 32) << 16);
+        const uint32_t s_addr = lane_addr + col_s(q), o_addr = lane_addr + col_o(q);
+        const uint32_t sQq = sQ + q * C::kTileBytes;
+        uint32_t gtt = 0;
         for (int it = 0;; ++it) {
             const int slot = it & 1;
             if (!wait_bar_warp(bar(B_ITEM_FULL + slot), (it >> 1) & 1, abort, hdr, 11)) break;
@@ -351,33 +374,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (item < 0) break;
             Item itm;
             decode(dv, BH, n_anchor, item, tile_off, qoff, qlist, itm);
+            if (q == 1 && itm.nq <= kQTile) continue;  // no tile B in this item
+            const int r_item = q * kQTile + row;       // row within the item
             const __nv_bfloat16* Qb = Q + size_t(itm.bh) * L * D;
-            // this thread's row: token and partial slot
             int my_tok = -1, my_slot = 0;
-            if (row < itm.nq) {
+            if (r_item < itm.nq) {
                 if (itm.slot_fixed >= 0) {
-                    my_tok = itm.q0 + row;
+                    my_tok = itm.q0 + r_item;
                 } else {
-                    const int e = itm.entries[row];
+                    const int e = itm.entries[r_item];
                     my_tok = e >> 5;
                     my_slot = 1 + (e & 31);
                 }
             }
-            // gather the warp's 32 query rows (2 rows x 16 B chunks per step)
-            constexpr int CH = D / 8;  // 16-byte chunks per row
+            // gather the warp's 32 query rows into the swizzled tile (16-byte chunks)
+            constexpr int CH = D / 8;
 #pragma unroll 4
-            for (int i = 0; i < 32 * CH / 32; ++i) {
+            for (int i = 0; i < CH; ++i) {
                 const int idx = i * 32 + lane;
-                const int r = warp * 32 + idx / CH, ch = idx % CH;
+                const int r = (warp & 3) * 32 + idx / CH, ch = idx % CH;
                 const int tok = __shfl_sync(0xffffffffu, my_tok, r & 31);
                 uint4 v = make_uint4(0, 0, 0, 0);
                 if (tok >= 0) v = ldg_nc16(Qb + size_t(tok) * D + ch * 8);
-                const uint32_t dst = sQ + (ch >> 3) * C::kSlabBytes + r * 128 + (((ch & 7) ^ (r & 7)) << 4);
+                const uint32_t dst = sQq + (ch >> 3) * C::kSlabBytes + r * 128 + (((ch & 7) ^ (r & 7)) << 4);
                 asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(v.x), "r"(v.y),
                              "r"(v.z), "r"(v.w) : "memory");
             }
             fence_proxy_async_smem();
-            mbar_arrive(bar(B_Q_FULL));
+            mbar_arrive(bar(B_Q_FULL + q));
 
             Cursor cur;
             cur.init(dv, itm);
@@ -386,16 +410,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; cur.more(); ++j) {
                 int key0, nvalid;
                 cur.next(key0, nvalid);
-                const uint32_t sb = gt & 1, n = gt >> 1;
-                if (!wait_bar_warp(bar(B_S_FULL + sb), n & 1, abort, hdr, 12)) { stop = true; break; }
+                if (!wait_bar_warp(bar(B_S_FULL + q), gtt & 1, abort, hdr, 12)) { stop = true; break; }
                 tc_fence_after();
                 uint32_t s[kKT];
 #pragma unroll
                 for (int c = 0; c < kKT / 32; ++c)
-                    tmem_ld32(lane_addr + sb * kKT + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
+                    tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
                 tmem_wait_ld();
-                tc_fence_before();
-                mbar_arrive(bar(B_S_FREE + sb));
                 // scale (log2 units), mask keys past the range end, row max
                 float mx = -INFINITY;
 #pragma unroll
@@ -413,22 +434,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     m_used = mx;
                     rescale = true;
                 }
-                float rs = 0.f;
-                uint32_t pk[kKT / 2];
-#pragma unroll
-                for (int c = 0; c < kKT; c += 2) {
-                    const float p0 = ex2(__uint_as_float(s[c]) - m_used);
-                    const float p1 = ex2(__uint_as_float(s[c + 1]) - m_used);
-                    rs += p0 + p1;
-                    pk[c / 2] = pack_bf16(p0, p1);
-                }
-                l = l * alpha + rs;
-                if (j > 0) {  // PV of the previous tile done: P buffer free, O current
-                    if (!wait_bar_warp(bar(B_P_FREE), (gt - 1) & 1, abort, hdr, 13)) { stop = true; break; }
-                    tc_fence_after();
-                }
                 if (__any_sync(0xffffffffu, rescale)) {  // warp-collective TMEM access; alpha = 1 elsewhere
-                    const uint32_t o_addr = lane_addr + 2 * kKT;
+                    // O_q must hold PV_q(j-1) before it is scaled
+                    if (!wait_bar_warp(bar(B_PV_DONE + q), (gtt - 1) & 1, abort, hdr, 13)) { stop = true; break; }
+                    tc_fence_after();
 #pragma unroll
                     for (int c = 0; c < D / 32; ++c) {
                         uint32_t o[32];
@@ -438,26 +447,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
                         tmem_st32(o_addr + c * 32, o);
                     }
-                    tmem_wait_st();
                 }
-                // P row -> shared memory, 128-byte swizzle (16 chunks of 8 keys)
+                // P = exp2(s - m) as bf16 pairs into the first 64 columns of S_q
+                float rs = 0.f;
 #pragma unroll
-                for (int ch = 0; ch < kKT / 8; ++ch) {
-                    const uint32_t dst = sP + (ch >> 3) * C::kSlabBytes + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
-                    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(pk[ch * 4]),
-                                 "r"(pk[ch * 4 + 1]), "r"(pk[ch * 4 + 2]), "r"(pk[ch * 4 + 3]) : "memory");
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const float p0 = ex2(__uint_as_float(s[h * 64 + 2 * c]) - m_used);
+                        const float p1 = ex2(__uint_as_float(s[h * 64 + 2 * c + 1]) - m_used);
+                        rs += p0 + p1;
+                        pk[c] = pack_bf16(p0, p1);
+                    }
+                    tmem_st32(s_addr + h * 32, pk);
                 }
-                fence_proxy_async_smem();
+                l = l * alpha + rs;
+                tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(bar(B_P_FULL));
-                ++gt;
+                mbar_arrive(bar(B_P_FULL + q));
+                ++gtt;
             }
             if (stop) break;
             // epilogue: final PV done -> O / l -> partial row, log-sum-exp
-            if (!wait_bar_warp(bar(B_P_FREE), (gt - 1) & 1, abort, hdr, 14)) break;
+            if (!wait_bar_warp(bar(B_PV_DONE + q), (gtt - 1) & 1, abort, hdr, 14)) break;
             tc_fence_after();
             const float inv = 1.f / l;
-            const uint32_t o_addr = lane_addr + 2 * kKT;
             float* dst = (my_tok >= 0) ? o_p + ((size_t(itm.bh) * L + my_tok) * S + my_slot) * D : nullptr;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
@@ -480,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }

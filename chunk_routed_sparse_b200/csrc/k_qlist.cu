@@ -4,7 +4,7 @@
 // This replaces the "pack every (query, key) group into one variable-length
 // attention call" step of the jxzklqfsx.com MoC write-up ("計算效率"): the
 // attention kernel walks chunk-major work items, each a chunk's keys against
-// up to 128 of the queries that selected it.
+// up to 256 of the queries that selected it.
 //
 // Entries are (query << 5 | slot), slot = position in sel. Every list is
 // sorted by query: each block owns kQlistBlock consecutive queries and one
@@ -37,7 +37,8 @@ __global__ void __launch_bounds__(32) qlist_count(int L, int C, int k, int nblk,
 }
 
 // Per (bh): blk_count -> exclusive offsets of each block within each chunk's
-// list (in place); qoff[bh*C + c] <- list length, tile_off[bh*C + c] <- tiles.
+// list (in place); qoff[bh*C + c] <- list length, tile_off[bh*C + c] <- attention
+// work items of kItemRows entries.
 __global__ void __launch_bounds__(256) qlist_scan_blocks(int C, int nblk,
                                                          int32_t* __restrict__ blk_count,
                                                          int32_t* __restrict__ qlen,
@@ -52,7 +53,7 @@ __global__ void __launch_bounds__(256) qlist_scan_blocks(int C, int nblk,
             run += v;
         }
         qlen[size_t(bh) * C + c] = run;
-        ntile[size_t(bh) * C + c] = (run + kQTile - 1) / kQTile;
+        ntile[size_t(bh) * C + c] = (run + kItemRows - 1) / kItemRows;
     }
 }
 

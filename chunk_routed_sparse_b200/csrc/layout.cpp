@@ -158,7 +158,7 @@ moc_status build_host(const moc_layout_desc* d, moc_layout* lay) {
         lay->rtile_off.push_back(lay->rtile_off.back() + (nq + moc::kQTile - 1) / moc::kQTile);
     }
     lay->total_rtiles = lay->rtile_off.back();
-    // anchor work items: groups with the most keys per tile first (longest work first)
+    // anchor work items of kItemRows queries: groups with the most keys first (longest work first)
     lay->a_order.resize(G);
     std::iota(lay->a_order.begin(), lay->a_order.end(), 0);
     std::stable_sort(lay->a_order.begin(), lay->a_order.end(),
@@ -167,7 +167,7 @@ moc_status build_host(const moc_layout_desc* d, moc_layout* lay) {
     for (int x = 0; x < G; ++x) {
         const int g = lay->a_order[x];
         const int32_t nq = lay->grp_q1[g] - lay->grp_q0[g];
-        lay->atile_off.push_back(lay->atile_off.back() + (nq + moc::kQTile - 1) / moc::kQTile);
+        lay->atile_off.push_back(lay->atile_off.back() + (nq + moc::kItemRows - 1) / moc::kItemRows);
     }
     lay->total_atiles = lay->atile_off.back();
     return MOC_OK;

@@ -10,7 +10,8 @@
 
 namespace moc {
 
-constexpr int kQTile = 128;       // query rows per router / attention work item
+constexpr int kQTile = 128;       // query rows per router tile and per attention MMA tile
+constexpr int kItemRows = 256;    // query rows per attention work item (two 128-row tiles)
 constexpr int kMaxK = 31;         // top-k limit: 1+k partial slots fit one warp
 constexpr int kMaxChunks = 16384; // chunk limit (query-list counters live in shared memory)
 constexpr int kQlistBlock = 1024; // queries per block of the query-list builder
@@ -28,7 +29,7 @@ struct DevLayout {
     const int32_t* cand;         // candidate chunk ids, ascending, per group
     const int32_t* cand_ncausal; // [G] length of the causal prefix of the list
     const int32_t* rtile_off;    // [G+1] prefix of router tiles (kQTile queries) per group
-    const int32_t* atile_off;    // [G+1] prefix of anchor tiles, groups in a_order
+    const int32_t* atile_off;    // [G+1] prefix of anchor items (kItemRows queries), groups in a_order
     const int32_t* a_order;      // [G] groups by descending anchor keys per tile
 };
 
@@ -56,7 +57,7 @@ struct WsPlan {
     size_t hdr = 0;        // int32[64]: [0] error code, [1] detail, [2] work counter
     size_t blk_count = 0;  // int32 [BH][nblk][C]
     size_t qoff = 0;       // int32 [BH*C + 1] global start of every list
-    size_t tile_off = 0;   // int32 [BH*C + 1] prefix of routed tiles
+    size_t tile_off = 0;   // int32 [BH*C + 1] prefix of routed items (kItemRows entries each)
     size_t qlist = 0;      // int32 [BH*L*k] entries (query << 5 | slot)
     size_t lse_p = 0;      // fp32 [BH][L][1+k]
     size_t o_p = 0;        // fp32 [BH][L][1+k][d]

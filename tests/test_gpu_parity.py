@@ -217,7 +217,7 @@ def test_qlists_invert_selection():
             assert np.all(s[bh, q, slot] == c)
             want = np.nonzero((s[bh] == c).any(-1))[0]
             assert np.array_equal(q, want)
-            assert tile[x + 1] - tile[x] == (len(ent) + 127) // 128
+            assert tile[x + 1] - tile[x] == (len(ent) + 255) // 256
 
 
 def test_deterministic_repeat():
