@@ -55,6 +55,7 @@ constexpr int kThreads = 384;                   // softmax A, softmax B, produce
 // the producer/MMA warpgroup drops to 72 and the softmax warpgroups rise to
 // 216: 2 x 128 x 216 + 128 x 72 = 64512, and per SM sub-partition
 // (one warp of each warpgroup) 32 x (216 + 216 + 72) = 16128 <= 16384.
+constexpr int kEmuEvery = 4;  // one exp2 pair in kEmuEvery on the FMA pipe (full tiles)
 constexpr int kRegsSoftmax = 216;
 constexpr int kRegsOther = 72;
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // bounded waits
@@ -417,14 +418,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < kKT / 32; ++c)
                     tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
                 tmem_wait_ld();
-                // scale (log2 units), mask keys past the range end, row max
-                float mx = -INFINITY;
+                // keys past the range end (only in a range's last tile) -> -inf, so P = 0
+                if (nvalid < kKT) {
 #pragma unroll
-                for (int c = 0; c < kKT; ++c) {
-                    const float v = (c < nvalid) ? __uint_as_float(s[c]) * scale_log2 : -INFINITY;
-                    s[c] = __float_as_uint(v);
-                    mx = fmaxf(mx, v);
+                    for (int c = 0; c < kKT; ++c)
+                        if (c >= nvalid) s[c] = __float_as_uint(-INFINITY);
                 }
+                // row max of the raw scores (the positive scale commutes with max)
+                float a0 = __uint_as_float(s[0]), a1 = __uint_as_float(s[1]);
+                float a2 = __uint_as_float(s[2]), a3 = __uint_as_float(s[3]);
+#pragma unroll
+                for (int c = 4; c < kKT; c += 8) {
+                    a0 = max3(a0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+                    a1 = max3(a1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+                    a2 = max3(a2, __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));
+                    a3 = max3(a3, __uint_as_float(s[c + 6]), __uint_as_float(s[c + 7]));
+                }
+                const float mx = max3(a0, a1, fmaxf(a2, a3)) * scale_log2;  // log2 units
                 float alpha = 1.f;
                 bool rescale = false;
                 if (j == 0) {
@@ -448,20 +458,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tmem_st32(o_addr + c * 32, o);
                     }
                 }
-                // P = exp2(s - m) as bf16 pairs into the first 64 columns of S_q
-                float rs = 0.f;
+                // P = exp2(s * scale - m) as bf16 pairs into the first 64 columns of S_q;
+                // scale-and-subtract and the row sum run on packed fp32 pairs
+                // (full tiles: every kEmuEvery-th pair on the FMA pipe, the rest on MUFU;
+                //  a range's last, masked tile: all on MUFU so masked keys give exactly 0)
+                const uint64_t sc2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m_used, -m_used);
+                const bool full = nvalid == kKT;
+                uint64_t sum2a = 0, sum2b = 0;
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     uint32_t pk[32];
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
-                        const float p0 = ex2(__uint_as_float(s[h * 64 + 2 * c]) - m_used);
-                        const float p1 = ex2(__uint_as_float(s[h * 64 + 2 * c + 1]) - m_used);
-                        rs += p0 + p1;
+                        const int e = h * 64 + 2 * c;
+                        float x0, x1, p0, p1;
+                        f2_unpack(f2_fma(f2_pack(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), sc2, nm2), x0, x1);
+                        if ((c % kEmuEvery) == kEmuEvery - 1 && full) {
+                            ex2_poly2(x0, x1, p0, p1);
+                        } else {
+                            p0 = ex2(x0);
+                            p1 = ex2(x1);
+                        }
+                        if (c & 1) sum2b = f2_add(sum2b, f2_pack(p0, p1));
+                        else sum2a = f2_add(sum2a, f2_pack(p0, p1));
                         pk[c] = pack_bf16(p0, p1);
                     }
                     tmem_st32(s_addr + h * 32, pk);
                 }
+                float r0, r1, r2, r3;
+                f2_unpack(sum2a, r0, r1);
+                f2_unpack(sum2b, r2, r3);
+                const float rs = (r0 + r1) + (r2 + r3);
                 l = l * alpha + rs;
                 tmem_wait_st();
                 tc_fence_before();
