@@ -18,8 +18,10 @@
 // 128-row tiles A and B that share one K/V stream:
 //   warp 8 (one lane): scheduler + TMA producer. Takes items from an atomic
 //          counter, publishes them in a 2-slot ring, streams 128-key K and V
-//          tiles (64-column, 128-byte-swizzled slabs) into a 2-stage ring with
-//          cp.async.bulk.tensor, completion counted on mbarriers.
+//          tiles (64-column, 128-byte-swizzled slabs) into 2-stage K and V rings
+//          with cp.async.bulk.tensor, completion counted on mbarriers. K(j) is
+//          released as soon as S(j) is computed, so K(j+2) loads while PV(j) and
+//          the next S still run.
 //          (warps 10-11 only complete the third warpgroup.)
 //   warp 9: allocates all 512 TMEM columns (S_A, S_B, O_A, O_B); one lane
 //          issues tcgen05.mma in the order
@@ -55,7 +57,6 @@ constexpr int kThreads = 384;                   // softmax A, softmax B, produce
 // the producer/MMA warpgroup drops to 72 and the softmax warpgroups rise to
 // 216: 2 x 128 x 216 + 128 x 72 = 64512, and per SM sub-partition
 // (one warp of each warpgroup) 32 x (216 + 216 + 72) = 16128 <= 16384.
-constexpr int kEmuEvery = 4;  // one exp2 pair in kEmuEvery on the FMA pipe (full tiles)
 constexpr int kRegsSoftmax = 216;
 constexpr int kRegsOther = 72;
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // bounded waits
@@ -82,8 +83,9 @@ __device__ __forceinline__ uint32_t col_o(int q) { return q ? 384u : 256u; }
 
 // mbarrier slots (8 bytes each) from Cfg::oBar; [x] = tile A / B or ring slot
 enum {
-    B_ITEM_FULL = 0, B_ITEM_EMPTY = 2, B_KV_FULL = 4, B_KV_EMPTY = 6, B_Q_FULL = 8,
-    B_S_FULL = 10, B_P_FULL = 12, B_PV_DONE = 14, B_MMA_DONE = 16, B_COUNT = 17
+    B_ITEM_FULL = 0, B_ITEM_EMPTY = 2, B_K_FULL = 4, B_K_EMPTY = 6, B_Q_FULL = 8,
+    B_S_FULL = 10, B_P_FULL = 12, B_PV_DONE = 14, B_V_FULL = 16, B_V_EMPTY = 18,
+    B_MMA_DONE = 20, B_COUNT = 21
 };
 
 struct Shared {  // at oBar + 192
@@ -222,8 +224,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int x = 0; x < 2; ++x) {
             mbar_init(bar(B_ITEM_FULL + x), 1);
             mbar_init(bar(B_ITEM_EMPTY + x), 1 + 256);
-            mbar_init(bar(B_KV_FULL + x), 1);
-            mbar_init(bar(B_KV_EMPTY + x), 1);
+            mbar_init(bar(B_K_FULL + x), 1);
+            mbar_init(bar(B_K_EMPTY + x), 1);
+            mbar_init(bar(B_V_FULL + x), 1);
+            mbar_init(bar(B_V_EMPTY + x), 1);
             mbar_init(bar(B_Q_FULL + x), 128);
             mbar_init(bar(B_S_FULL + x), 1);
             mbar_init(bar(B_P_FULL + x), 128);
@@ -268,24 +272,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                 while (cur.more()) {
                     int key0, nvalid;
                     cur.next(key0, nvalid);
+                    // K and V have rings of their own: K(j) is released once S(j) is computed,
+                    // long before V(j) is released by PV(j), so K(j+2) streams in early
                     const int st = gt & 1;
-                    if (!wait_bar(bar(B_KV_EMPTY + st), ((gt >> 1) & 1) ^ 1, abort, hdr, 2)) { stop = true; break; }
-                    mbar_expect_tx(bar(B_KV_FULL + st), 2 * C::kTileBytes);
+                    const uint32_t par = ((gt >> 1) & 1) ^ 1;
+                    if (!wait_bar(bar(B_K_EMPTY + st), par, abort, hdr, 2)) { stop = true; break; }
+                    mbar_expect_tx(bar(B_K_FULL + st), C::kTileBytes);
 #pragma unroll
-                    for (int s = 0; s < C::kSlabs; ++s) {
-                        tma_load_2d(sK + st * C::kTileBytes + s * C::kSlabBytes, &tmK, bar(B_KV_FULL + st), 64 * s, row0 + key0);
-                        tma_load_2d(sV + st * C::kTileBytes + s * C::kSlabBytes, &tmV, bar(B_KV_FULL + st), 64 * s, row0 + key0);
-                    }
+                    for (int s = 0; s < C::kSlabs; ++s)
+                        tma_load_2d(sK + st * C::kTileBytes + s * C::kSlabBytes, &tmK, bar(B_K_FULL + st), 64 * s, row0 + key0);
+                    if (!wait_bar(bar(B_V_EMPTY + st), par, abort, hdr, 8)) { stop = true; break; }
+                    mbar_expect_tx(bar(B_V_FULL + st), C::kTileBytes);
+#pragma unroll
+                    for (int s = 0; s < C::kSlabs; ++s)
+                        tma_load_2d(sV + st * C::kTileBytes + s * C::kSlabBytes, &tmV, bar(B_V_FULL + st), 64 * s, row0 + key0);
                     ++gt;
                 }
                 if (stop) break;
             }
-            // drain: the last use of each stage has landed before the CTA exits
+            // drain: the last use of each stage has landed before the CTA exits (a load
+            // cut short by an abort may have issued K without V; its V wait then times out
+            // harmlessly because nothing was issued on it)
             for (uint32_t g = (gt >= 2 ? gt - 2 : 0); g < gt; ++g) {
                 const uint32_t st = g & 1, par = (g >> 1) & 1;
-                const uint64_t t0 = globaltimer();
-                while (!mbar_try_wait(bar(B_KV_FULL + st), par)) {
-                    if (globaltimer() - t0 > kTimeoutNs) { set_error(hdr, ERR_TIMEOUT, 9); break; }
+                for (int b = 0; b < 2; ++b) {
+                    const uint64_t t0 = globaltimer();
+                    while (!mbar_try_wait(bar((b ? B_V_FULL : B_K_FULL) + st), par)) {
+                        if (globaltimer() - t0 > kTimeoutNs) { set_error(hdr, ERR_TIMEOUT, 9); break; }
+                    }
                 }
             }
         }
@@ -313,10 +327,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 for (int j = 0; j <= T && !stop; ++j) {
                     const uint32_t st = gt & 1;
-                    bool kv_ready = false;
+                    bool k_ready = false, v_ready = false;
                     for (int q = 0; q < nt; ++q) {
                         if (j > 0) {  // O_q += P_q(j-1) V(j-1)
                             const uint32_t g = gtt[q] - 1, pst = (gt - 1) & 1;
+                            if (!v_ready) {
+                                if (!wait_bar(bar(B_V_FULL + pst), ((gt - 1) >> 1) & 1, abort, hdr, 15)) { stop = true; break; }
+                                v_ready = true;
+                            }
                             if (!wait_bar(bar(B_P_FULL + q), g & 1, abort, hdr, 7)) { stop = true; break; }
                             tc_fence_after();
 #pragma unroll
@@ -327,9 +345,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             umma_commit(bar(B_PV_DONE + q));
                         }
                         if (j < T) {  // S_q(j) = Q_q K(j)^T, after PV_q(j-1) has read P_q(j-1)
-                            if (!kv_ready) {
-                                if (!wait_bar(bar(B_KV_FULL + st), (gt >> 1) & 1, abort, hdr, 5)) { stop = true; break; }
-                                kv_ready = true;
+                            if (!k_ready) {
+                                if (!wait_bar(bar(B_K_FULL + st), (gt >> 1) & 1, abort, hdr, 5)) { stop = true; break; }
+                                k_ready = true;
                                 tc_fence_after();
                             }
                             const uint32_t qb = sQ + q * C::kTileBytes, kb = sK + st * C::kTileBytes;
@@ -344,7 +362,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                     if (stop) break;
-                    if (j > 0) umma_commit(bar(B_KV_EMPTY + ((gt - 1) & 1)));  // K(j-1), V(j-1) read
+                    if (j > 0) umma_commit(bar(B_V_EMPTY + ((gt - 1) & 1)));  // V(j-1) read by PV
+                    if (j < T) umma_commit(bar(B_K_EMPTY + st));              // K(j) read by S
                     if (j < T) ++gt;
                 }
                 for (int q = 0; q < nt; ++q) ++itq[q];
@@ -460,10 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 // P = exp2(s * scale - m) as bf16 pairs into the first 64 columns of S_q;
                 // scale-and-subtract and the row sum run on packed fp32 pairs
-                // (full tiles: every kEmuEvery-th pair on the FMA pipe, the rest on MUFU;
-                //  a range's last, masked tile: all on MUFU so masked keys give exactly 0)
                 const uint64_t sc2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m_used, -m_used);
-                const bool full = nvalid == kKT;
                 uint64_t sum2a = 0, sum2b = 0;
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
@@ -471,14 +487,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
                         const int e = h * 64 + 2 * c;
-                        float x0, x1, p0, p1;
+                        float x0, x1;
                         f2_unpack(f2_fma(f2_pack(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), sc2, nm2), x0, x1);
-                        if ((c % kEmuEvery) == kEmuEvery - 1 && full) {
-                            ex2_poly2(x0, x1, p0, p1);
-                        } else {
-                            p0 = ex2(x0);
-                            p1 = ex2(x1);
-                        }
+                        const float p0 = ex2(x0), p1 = ex2(x1);
                         if (c & 1) sum2b = f2_add(sum2b, f2_pack(p0, p1));
                         else sum2a = f2_add(sum2a, f2_pack(p0, p1));
                         pk[c] = pack_bf16(p0, p1);

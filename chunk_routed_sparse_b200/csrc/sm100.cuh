@@ -184,35 +184,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
     return d;
 }
 
-// 2^x for a pair of finite x <= 8 on the FMA/ALU pipes instead of the MUFU
-// unit. Method: round x to the nearest integer j by adding 1.5 * 2^23 (the
-// sum's low mantissa bits hold j), f = x - j in [-1/2, 1/2], 2^f by a degree-3
-// polynomial (Horner), and 2^j applied by adding j << 23 to the exponent
-// field. The coefficients are the minimax fit of 2^f on [-1/2, 1/2] under
-// relative error (a linear program on a dense grid), max relative error
-// 7.5e-5 in fp32 evaluation. x is clamped at -125 so that the result stays a
-// normal number (a contribution below 2^-125 is negligible).
-constexpr float kExp2C0 = 0.9999279975891113f;
-constexpr float kExp2C1 = 0.6932609677314758f;
-constexpr float kExp2C2 = 0.2426113784313202f;
-constexpr float kExp2C3 = 0.05517177656292915f;
-__device__ __forceinline__ void ex2_poly2(float x0, float x1, float& y0, float& y1) {
-    const float kMagic = 12582912.0f;  // 1.5 * 2^23
-    const uint64_t x = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-    const uint64_t t = f2_add(x, f2_pack(kMagic, kMagic));
-    const uint64_t j = f2_add(t, f2_pack(-kMagic, -kMagic));
-    const uint64_t f = f2_fma(j, f2_pack(-1.f, -1.f), x);
-    uint64_t p = f2_fma(f, f2_pack(kExp2C3, kExp2C3), f2_pack(kExp2C2, kExp2C2));
-    p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
-    p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
-    float p0, p1, t0, t1;
-    f2_unpack(p, p0, p1);
-    f2_unpack(t, t0, t1);
-    // t's bits are 0x4B400000 + j, and 0x4B400000 << 23 vanishes mod 2^32
-    y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-    y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
-}
-
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
