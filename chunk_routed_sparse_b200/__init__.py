@@ -67,6 +67,7 @@ SIGNATURES = {
     "moc_attention_fwd": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _F, _P, _P, _P, _SZ, _P]),
     "moc_attention_fwd_static": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _F, _P, _P, _P]),
     "moc_check_device_error": (_I, [_P, _SZ, _P, _P]),
+    "moc_layout_device_error": (_I, [_P, _P, _P]),
 }
 
 
@@ -238,6 +239,14 @@ def forward(layout: Layout, Q, K, V, k: int, causal: bool = True, scale=None, ws
         torch.empty(Q.shape[0], Q.shape[1], Q.shape[2], 0, dtype=torch.int32, device=Q.device)
     O, lse = attention_fwd(layout, Q, K, V, sel, k, scale=scale, ws=ws)
     return O, lse, sel, kbar
+
+
+def check_layout_error(layout: Layout) -> int:
+    """Read and clear the layout's device error word (router); raises on error."""
+    det = ctypes.c_int32()
+    _check(lib().moc_layout_device_error(layout.handle, ctypes.byref(det), _stream()),
+           "layout device error word")
+    return det.value
 
 
 def check_device_error(ws: torch.Tensor) -> int:

@@ -41,10 +41,8 @@
 // Every mbarrier wait is bounded (2 s): on timeout the kernel records
 // ERR_TIMEOUT and a site code in the workspace header, every role leaves its
 // loop, in-flight copies and MMAs are drained (bounded) and TMEM is freed.
-#include <cuda.h>
-
-#include "common.cuh"
-#include "sm100.cuh"
+#include "pipeline.cuh"
+#include "tmap.cuh"
 
 namespace moc {
 namespace {
@@ -59,7 +57,6 @@ constexpr int kThreads = 384;                   // softmax A, softmax B, produce
 // (one warp of each warpgroup) 32 x (216 + 216 + 72) = 16128 <= 16384.
 constexpr int kRegsSoftmax = 216;
 constexpr int kRegsOther = 72;
-constexpr uint64_t kTimeoutNs = 2000000000ull;  // bounded waits
 constexpr uint32_t kTmemCols = 512;
 
 template <int D>
@@ -168,32 +165,6 @@ __device__ __forceinline__ int count_tiles(const DevLayout& dv, const Item& it) 
     int t = 0;
     for (int r = it.r_beg; r < it.r_end; ++r) t += (dv.ar[2 * r + 1] - dv.ar[2 * r] + kKT - 1) / kKT;
     return t;
-}
-
-// Bounded wait; false on timeout or when another role aborted.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort,
-                                         int32_t* hdr, int where) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer();
-    for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63) == 0) {
-            if (*abort) return false;
-            if (globaltimer() - t0 > kTimeoutNs) {
-                set_error(hdr, ERR_TIMEOUT, where);
-                *abort = 1;
-                return false;
-            }
-        }
-    }
-}
-
-// The same wait, made uniform across the warp (the softmax warps execute
-// warp-collective tcgen05.ld/st right after it).
-__device__ __forceinline__ bool wait_bar_warp(uint32_t bar, uint32_t parity, volatile int* abort,
-                                              int32_t* hdr, int where) {
-    const bool ok = wait_bar(bar, parity, abort, hdr, where);
-    return __all_sync(0xffffffffu, ok);
 }
 
 template <int D>
@@ -537,36 +508,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
-}
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
-// [rows][d] bf16 matrix, box = 64 columns (128 B) x 128 rows, 128-byte swizzle
-bool make_tmap(CUtensorMap* tm, const void* ptr, int d, int64_t rows) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(rows)};
-    cuuint64_t strides[1] = {cuuint64_t(d) * 2};
-    cuuint32_t box[2] = {64, 128};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int D>

@@ -1,4 +1,5 @@
-// (2) Router: per-query top-k over candidate chunks.
+// (2) Router: per-query top-k over candidate chunks, on the tcgen05 tensor
+// cores.
 //
 // "Mixture of Contexts for Long Video Generation | Summary" §3.1: each query
 // scores candidate chunks by the dot product with their mean-pooled keys and
@@ -7,202 +8,350 @@
 // "計算效率": mandatory chunks are inserted before top-k so that the router
 // spends no budget on them (they are not candidates).
 //
-// One CTA per (b*h, 128-query tile of one query group). All queries of a
-// group share one candidate list. Per block of 64 candidates:
-//   * the fp32 pooled keys are split into hi + lo bf16 parts (hi = RN(x),
-//     lo = RN(x - hi)); Q is exactly bf16, so q.hi + q.lo on the tensor cores
-//     (mma.sync m16n8k16, fp32 accumulate) reproduces q.Kbar to about 2^-17
-//     relative per term instead of bf16's 2^-9;
-//   * the 128 x 64 scores go to shared memory and every query row is scanned
-//     by two threads (32 candidates each), each keeping a sorted top-KMAX list
-//     in registers (KMAX: compile-time bound >= k). The two lists are merged
-//     at the end. Ties rank the lower chunk id first.
-#include "common.cuh"
+// Work unit: a 128-query tile of one query group (all its queries share one
+// candidate list) times a block of <= 256 of the group's candidates. One
+// persistent CTA per SM walks a contiguous range of tiles, 320 threads:
+//   warp 8 (one lane): streams each tile's Q rows (two 64-column,
+//          128-byte-swizzled slabs) into a 2-stage ring with TMA;
+//   warp 9: owns 512 TMEM columns (one 256-column score buffer per selection
+//          warpgroup). When the (head, group, block) changes it converts the
+//          block's fp32 pooled keys into swizzled bf16 operands hi = RN(Kbar)
+//          and lo = RN(Kbar - hi) - Q is exact bf16, so the two bf16 products
+//          reproduce q . Kbar to ~2^-17 relative per term - and its lane 0
+//          issues S = Q hi^T + Q lo^T (M=128, N = block rounded up to 16,
+//          K = d, fp32 accumulation in TMEM);
+//   warps 0-3 / 4-7: two selection warpgroups taking alternate tiles; one
+//          thread per query row (= TMEM lane) reads its scores from TMEM and
+//          keeps a sorted top-KMAX list in registers with a branch-free
+//          insertion network (candidates come in ascending id, so a strict
+//          ">" orders ties by lower chunk id), writing the first k entries
+//          (-1 padded) after the tile's last block.
+// Tiles without candidates (caption groups, the first shot) are written as -1
+// rows by their selection warpgroup and skip the other roles. Waits are
+// bounded as in the attention kernel; a timeout is recorded in the layout's
+// device error word.
+#include "pipeline.cuh"
+#include "tmap.cuh"
 
 namespace moc {
 namespace {
 
-constexpr int kCandBlock = 64;
+using namespace sm100;
+
+constexpr int kBlk = 256;  // candidates per MMA block (N <= 256)
 constexpr int kIdNone = 0x7fffffff;
+constexpr int kRThreads = 320;
 
 template <int D>
-struct RouteSmem {
-    static constexpr int kStride = D + 8;  // bf16 elements per row (+16 B: conflict-free fragments)
-    static constexpr int kSStride = kCandBlock + 1;  // odd pitch: row-per-thread scans are conflict-free
-    __nv_bfloat16 q[kQTile][kStride];
-    __nv_bfloat16 khi[kCandBlock][kStride];
-    __nv_bfloat16 klo[kCandBlock][kStride];
-    float s[kQTile][kSStride];
-    int cid[kCandBlock];
+struct RCfg {
+    static constexpr int kSlabs = D / 64;
+    static constexpr int kQBytes = kSlabs * 128 * 128;  // one 128-row Q tile
+    static constexpr int kKbSlab = kBlk * 128;          // 256 rows x 128 B
+    static constexpr int kKbBytes = kSlabs * kKbSlab;   // hi (or lo) block
+    static constexpr int oQ = 0;                        // 2 stages
+    static constexpr int oHi = oQ + 2 * kQBytes;
+    static constexpr int oLo = oHi + kKbBytes;
+    static constexpr int oBar = oLo + kKbBytes;
+    static constexpr int kSmem = (oBar + 256 + 1024) > 120 * 1024 ? (oBar + 256 + 1024) : 120 * 1024;
 };
 
-// Insert (cs, cj) into a sorted (best first) register list of KMAX entries
-// if it ranks before the last entry; the last entry drops out.
-template <int KMAX>
-__device__ __forceinline__ void topk_insert(float (&ts)[KMAX], int (&tj)[KMAX], float cs, int cj) {
-    if (!ranks_before(cs, cj, ts[KMAX - 1], tj[KMAX - 1])) return;
-    ts[KMAX - 1] = cs;
-    tj[KMAX - 1] = cj;
-#pragma unroll
-    for (int x = KMAX - 1; x > 0; --x) {
-        if (ranks_before(ts[x], tj[x], ts[x - 1], tj[x - 1])) {
-            const float fs = ts[x]; ts[x] = ts[x - 1]; ts[x - 1] = fs;
-            const int fj = tj[x]; tj[x] = tj[x - 1]; tj[x - 1] = fj;
-        }
-    }
-}
+// R_S_FULL / R_S_FREE: [warpgroup]; R_KB_FREE: the MMAs that read the operand block are done
+enum { R_Q_FULL = 0, R_Q_EMPTY = 2, R_S_FULL = 4, R_S_FREE = 6, R_KB_FREE = 8, R_MMA_DONE = 9 };
 
-template <int D, int KMAX>
-__global__ void __launch_bounds__(256, KMAX <= 16 ? 2 : 1)
-    route_kernel(DevLayout dv, const __nv_bfloat16* __restrict__ Q, const float* __restrict__ Kbar,
-                 int k, int causal, int32_t* __restrict__ sel) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    RouteSmem<D>& sm = *reinterpret_cast<RouteSmem<D>*>(smem_raw);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.y;
-    const int tile = blockIdx.x;
-    const int g = upper_index(dv.rtile_off, dv.G + 1, tile);
-    const int q0 = dv.grp_q0[g] + (tile - dv.rtile_off[g]) * kQTile;
-    const int nq = min(kQTile, dv.grp_q1[g] - q0);
-    int32_t* out = sel + (size_t(bh) * dv.L + q0) * k;
-    const int cbeg = dv.cand_off[g];
-    const int ncand = (dv.grp_kind[g] != MOC_VIDEO) ? 0
-                      : causal ? dv.cand_ncausal[g] : dv.cand_off[g + 1] - cbeg;
-    if (ncand == 0) {
-        for (int i = tid; i < nq * k; i += blockDim.x) out[i] = -1;
-        return;
-    }
-    // query tile -> shared memory (rows past the group end are zero)
-    constexpr int V8 = D / 8;
-    const __nv_bfloat16* qsrc = Q + (size_t(bh) * dv.L + q0) * D;
-    for (int i = tid; i < kQTile * V8; i += blockDim.x) {
-        const int r = i / V8, c = i % V8;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (r < nq) v = ldg_nc16(qsrc + size_t(r) * D + c * 8);
-        *reinterpret_cast<uint4*>(&sm.q[r][c * 8]) = v;
-    }
-    float ts[KMAX];
-    int tj[KMAX];
+struct RShared {  // at oBar + 128
+    uint32_t tmem_base;
+    int abort;
+};
+
+// Insert (cs, cj) into a register list sorted by descending score (branch
+// free: one compare and four selects per entry). Candidates arrive in
+// ascending chunk id, so the strict ">" keeps an equal score behind the
+// earlier, lower id - the list is ordered by (score desc, id asc) without
+// ever comparing ids. The last entry drops out.
+template <int KMAX>
+__device__ __forceinline__ void topk_push(float (&ts)[KMAX], int (&tj)[KMAX], float cs, int cj) {
 #pragma unroll
     for (int x = 0; x < KMAX; ++x) {
-        ts[x] = -INFINITY;
-        tj[x] = kIdNone;
+        const bool gt = cs > ts[x];
+        const float ks = gt ? cs : ts[x];
+        const int kj = gt ? cj : tj[x];
+        cs = gt ? ts[x] : cs;
+        cj = gt ? tj[x] : cj;
+        ts[x] = ks;
+        tj[x] = kj;
     }
-    const int row = tid & (kQTile - 1), half = tid >> 7;
-    const int g8 = lane >> 2, t4 = lane & 3;
+}
+
+struct Tile {
+    int bh, g, q0, nq, cbeg, ncand, nb;
+};
+
+__device__ __forceinline__ void decode_tile(const DevLayout& dv, int64_t rtiles, int causal, int64_t t,
+                                            Tile& x) {
+    x.bh = int(t / rtiles);
+    const int rt = int(t % rtiles);
+    x.g = upper_index(dv.rtile_off, dv.G + 1, rt);
+    x.q0 = dv.grp_q0[x.g] + (rt - dv.rtile_off[x.g]) * kQTile;
+    x.nq = min(kQTile, dv.grp_q1[x.g] - x.q0);
+    x.cbeg = dv.cand_off[x.g];
+    x.ncand = (dv.grp_kind[x.g] != MOC_VIDEO) ? 0
+              : causal ? dv.cand_ncausal[x.g] : dv.cand_off[x.g + 1] - x.cbeg;
+    x.nb = (x.ncand + kBlk - 1) / kBlk;
+}
+
+// Fill the hi / lo operand block (K-major, 128-byte swizzle) of candidates
+// [cbeg + b * kBlk, + nbc) of head bh; rows up to npad are zero. Run by one warp.
+template <int D, int KBSLAB>
+__device__ __forceinline__ void build_block(const DevLayout& dv, const float* __restrict__ Kbar, int bh, int cbeg,
+                                            int b, int nbc, int npad, uint32_t sHi, uint32_t sLo, int lane) {
     const float* kb = Kbar + size_t(bh) * dv.C * D;
-    for (int cb = 0; cb < ncand; cb += kCandBlock) {
-        __syncthreads();  // previous block's candidates and scores fully consumed
-        constexpr int V4 = D / 4;
-        for (int i = tid; i < kCandBlock * V4; i += blockDim.x) {
-            const int r = i / V4, c = i % V4;
-            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (cb + r < ncand)
-                x = *reinterpret_cast<const float4*>(kb + size_t(dv.cand[cbeg + cb + r]) * D + c * 4);
-            __nv_bfloat162 h01 = __floats2bfloat162_rn(x.x, x.y);
-            __nv_bfloat162 h23 = __floats2bfloat162_rn(x.z, x.w);
-            float2 f01 = __bfloat1622float2(h01), f23 = __bfloat1622float2(h23);
-            __nv_bfloat162 l01 = __floats2bfloat162_rn(x.x - f01.x, x.y - f01.y);
-            __nv_bfloat162 l23 = __floats2bfloat162_rn(x.z - f23.x, x.w - f23.y);
-            *reinterpret_cast<__nv_bfloat162*>(&sm.khi[r][c * 4]) = h01;
-            *reinterpret_cast<__nv_bfloat162*>(&sm.khi[r][c * 4 + 2]) = h23;
-            *reinterpret_cast<__nv_bfloat162*>(&sm.klo[r][c * 4]) = l01;
-            *reinterpret_cast<__nv_bfloat162*>(&sm.klo[r][c * 4 + 2]) = l23;
+    constexpr int CH = D / 8;  // 16-byte output chunks (8 dims) per row
+    for (int i = lane; i < npad * CH; i += 32) {
+        const int r = i / CH, ch = i % CH;
+        float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        if (r < nbc) {
+            const int c = dv.cand[cbeg + b * kBlk + r];
+            const float4 a = *reinterpret_cast<const float4*>(kb + size_t(c) * D + ch * 8);
+            const float4 bq = *reinterpret_cast<const float4*>(kb + size_t(c) * D + ch * 8 + 4);
+            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+            v[4] = bq.x; v[5] = bq.y; v[6] = bq.z; v[7] = bq.w;
         }
-        if (tid < kCandBlock) sm.cid[tid] = (cb + tid < ncand) ? dv.cand[cbeg + cb + tid] : kIdNone;
-        __syncthreads();
-
-        // scores of this warp's 16 queries x 64 candidates
-        float acc[8][4];
+        uint32_t hi[4], lo[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-        const int qr = warp * 16;
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-            const int k0 = ks * 16;
-            uint32_t a[4];
-            a[0] = *reinterpret_cast<const uint32_t*>(&sm.q[qr + g8][k0 + 2 * t4]);
-            a[1] = *reinterpret_cast<const uint32_t*>(&sm.q[qr + g8 + 8][k0 + 2 * t4]);
-            a[2] = *reinterpret_cast<const uint32_t*>(&sm.q[qr + g8][k0 + 8 + 2 * t4]);
-            a[3] = *reinterpret_cast<const uint32_t*>(&sm.q[qr + g8 + 8][k0 + 8 + 2 * t4]);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int n = j * 8 + g8;
-                uint32_t h0 = *reinterpret_cast<const uint32_t*>(&sm.khi[n][k0 + 2 * t4]);
-                uint32_t h1 = *reinterpret_cast<const uint32_t*>(&sm.khi[n][k0 + 8 + 2 * t4]);
-                uint32_t l0 = *reinterpret_cast<const uint32_t*>(&sm.klo[n][k0 + 2 * t4]);
-                uint32_t l1 = *reinterpret_cast<const uint32_t*>(&sm.klo[n][k0 + 8 + 2 * t4]);
-                mma_bf16_16816(acc[j], a, h0, h1);
-                mma_bf16_16816(acc[j], a, l0, l1);
-            }
+        for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+            const float2 hf = __bfloat1622float2(h);
+            const __nv_bfloat162 l2 = __floats2bfloat162_rn(v[2 * e] - hf.x, v[2 * e + 1] - hf.y);
+            hi[e] = *reinterpret_cast<const uint32_t*>(&h);
+            lo[e] = *reinterpret_cast<const uint32_t*>(&l2);
         }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            sm.s[qr + g8][j * 8 + 2 * t4] = acc[j][0];
-            sm.s[qr + g8][j * 8 + 2 * t4 + 1] = acc[j][1];
-            sm.s[qr + g8 + 8][j * 8 + 2 * t4] = acc[j][2];
-            sm.s[qr + g8 + 8][j * 8 + 2 * t4 + 1] = acc[j][3];
-        }
-        __syncthreads();
-
-        // each thread scans 32 candidates of its row
-        const int nblk = min(kCandBlock, ncand - cb);
-        const int c1 = min(nblk, half * 32 + 32);
-        for (int c = half * 32; c < c1; ++c) topk_insert<KMAX>(ts, tj, sm.s[row][c], sm.cid[c]);
-    }
-    // merge the two halves of every row: half 1 publishes, half 0 merges
-    __syncthreads();
-    float* pub_s = &sm.s[0][0];
-    int* pub_j = reinterpret_cast<int*>(&sm.q[0][0]);  // q is no longer read
-    if (half == 1) {
-#pragma unroll
-        for (int x = 0; x < KMAX; ++x) {
-            pub_s[row * KMAX + x] = ts[x];
-            pub_j[row * KMAX + x] = tj[x];
-        }
-    }
-    __syncthreads();
-    if (half == 0) {
-#pragma unroll
-        for (int x = 0; x < KMAX; ++x) topk_insert<KMAX>(ts, tj, pub_s[row * KMAX + x], pub_j[row * KMAX + x]);
-        if (row < nq) {
-            int32_t* o = out + size_t(row) * k;
-#pragma unroll
-            for (int x = 0; x < KMAX; ++x)
-                if (x < k) o[x] = (tj[x] == kIdNone) ? -1 : tj[x];
-        }
+        const uint32_t off = (ch >> 3) * KBSLAB + r * 128 + (((ch & 7) ^ (r & 7)) << 4);
+        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(sHi + off), "r"(hi[0]), "r"(hi[1]),
+                     "r"(hi[2]), "r"(hi[3]) : "memory");
+        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(sLo + off), "r"(lo[0]), "r"(lo[1]),
+                     "r"(lo[2]), "r"(lo[3]) : "memory");
     }
 }
 
 template <int D, int KMAX>
-cudaError_t launch_route_dk(const DevLayout& dv, int BH, int64_t rtiles, const void* Q,
-                            const float* Kbar, int k, int causal, int32_t* sel, cudaStream_t s) {
-    const int smem = int(sizeof(RouteSmem<D>));
-    cudaError_t e = cudaFuncSetAttribute(route_kernel<D, KMAX>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+__global__ void __launch_bounds__(kRThreads, 1)
+    route_tc_kernel(const __grid_constant__ CUtensorMap tmQ, DevLayout dv, int64_t total_tiles,
+                    int64_t rtiles, const float* __restrict__ Kbar, int k, int causal,
+                    int32_t* __restrict__ sel) {
+    using C = RCfg<D>;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    unsigned char* gbase = smem_raw + (base - raw);
+    const uint32_t sQ = base + C::oQ, sHi = base + C::oHi, sLo = base + C::oLo;
+    const uint32_t sBar = base + C::oBar;
+    RShared& sh = *reinterpret_cast<RShared*>(gbase + C::oBar + 128);
+    volatile int* abort = &sh.abort;
+    int32_t* err = dv.err;
+    auto bar = [&](int i) { return sBar + 8u * uint32_t(i); };
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    // this CTA's contiguous range of tiles
+    const int64_t t_beg = total_tiles * blockIdx.x / gridDim.x;
+    const int64_t t_end = total_tiles * (blockIdx.x + 1) / gridDim.x;
+
+    if (tid == 0) {
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(bar(R_Q_FULL + x), 1);
+            mbar_init(bar(R_Q_EMPTY + x), 1);
+            mbar_init(bar(R_S_FULL + x), 1);
+            mbar_init(bar(R_S_FREE + x), 128);
+        }
+        mbar_init(bar(R_KB_FREE), 1);
+        mbar_init(bar(R_MMA_DONE), 1);
+        sh.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 9) {
+        tmem_alloc(smem_u32(&sh.tmem_base), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sh.tmem_base;
+
+    if (warp == 8) {
+        // ------------------------------------------------------------ Q producer
+        if (lane == 0) {
+            prefetch_tmap(&tmQ);
+            uint32_t qi = 0;
+            for (int64_t t = t_beg; t < t_end; ++t) {
+                Tile x;
+                decode_tile(dv, rtiles, causal, t, x);
+                if (x.ncand == 0) continue;
+                const int st = qi & 1;
+                if (!wait_bar(bar(R_Q_EMPTY + st), ((qi >> 1) & 1) ^ 1, abort, err, 21)) break;
+                mbar_expect_tx(bar(R_Q_FULL + st), C::kQBytes);
+#pragma unroll
+                for (int s = 0; s < C::kSlabs; ++s)
+                    tma_load_2d(sQ + st * C::kQBytes + s * 128 * 128, &tmQ, bar(R_Q_FULL + st), 64 * s,
+                                x.bh * dv.L + x.q0);
+                ++qi;
+            }
+            // outstanding loads land before the CTA exits
+            for (uint32_t g = (qi >= 2 ? qi - 2 : 0); g < qi; ++g)
+                drain_bar(bar(R_Q_FULL + (g & 1)), (g >> 1) & 1, err, 29);
+        }
+        __syncwarp();
+    } else if (warp == 9) {
+        // ------------------------------------------------------------ operands + MMA issue
+        // The whole warp walks the units; it rebuilds the hi / lo block when the
+        // (head, group, block) changes - after the MMAs that read the old block
+        // have completed - and lane 0 issues the MMAs into the score buffer of
+        // the warpgroup that owns the tile (tiles alternate between the two).
+        uint32_t qi = 0, nkb = 0, uw[2] = {0, 0};
+        int last_bh = -1, last_g = -1, last_b = -1, ti = 0;
+        bool stop = false;
+        for (int64_t t = t_beg; t < t_end && !stop; ++t, ++ti) {
+            Tile x;
+            decode_tile(dv, rtiles, causal, t, x);
+            if (x.ncand == 0) continue;
+            const int w = ti & 1;
+            const int st = qi & 1;
+            if (!wait_bar_warp(bar(R_Q_FULL + st), (qi >> 1) & 1, abort, err, 22)) break;
+            for (int b = 0; b < x.nb; ++b) {
+                const int nbc = min(kBlk, x.ncand - b * kBlk);
+                const int npad = (nbc + 15) & ~15;
+                if (x.bh != last_bh || x.g != last_g || b != last_b) {
+                    if (last_bh >= 0) {  // the previous block's MMAs are complete
+                        if (lane == 0) umma_commit(bar(R_KB_FREE));
+                        if (!wait_bar_warp(bar(R_KB_FREE), nkb & 1, abort, err, 23)) { stop = true; break; }
+                        ++nkb;
+                    }
+                    build_block<D, C::kKbSlab>(dv, Kbar, x.bh, x.cbeg, b, nbc, npad, sHi, sLo, lane);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    last_bh = x.bh; last_g = x.g; last_b = b;
+                }
+                // one score buffer per warpgroup: its n-th use waits for the (n-1)-th release
+                if (!wait_bar_warp(bar(R_S_FREE + w), (uw[w] & 1) ^ 1, abort, err, 24)) { stop = true; break; }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t idesc = idesc_bf16_f32(128, npad, 0);
+                    const uint32_t d_s = tmem + w * 256;
+#pragma unroll
+                    for (int kk = 0; kk < 2 * (D / 16); ++kk) {  // hi then lo
+                        const int kd = kk % (D / 16);
+                        const uint32_t qoff = (kd >> 2) * 128 * 128 + (kd & 3) * 32;
+                        const uint32_t boff = (kd >> 2) * C::kKbSlab + (kd & 3) * 32;
+                        umma_ss(d_s, sdesc_sw128(sQ + st * C::kQBytes + qoff, 16, 1024),
+                                sdesc_sw128((kk < D / 16 ? sHi : sLo) + boff, 16, 1024), idesc, kk > 0);
+                    }
+                    umma_commit(bar(R_S_FULL + w));
+                }
+                __syncwarp();
+                ++uw[w];
+            }
+            if (stop) break;
+            if (lane == 0) umma_commit(bar(R_Q_EMPTY + st));
+            __syncwarp();
+            ++qi;
+        }
+        if (lane == 0) {
+            umma_commit(bar(R_MMA_DONE));
+            drain_bar(bar(R_MMA_DONE), 0, err, 30);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ selection (warpgroups 0, 1)
+        const int w = warp >> 2;        // this warpgroup takes tiles ti with ti % 2 == w
+        const int row = tid & 127;      // TMEM lane
+        const uint32_t lane_addr = tmem + (uint32_t((warp & 3) * 32) << 16) + w * 256;
+        uint32_t u = 0;
+        int ti = 0;
+        for (int64_t t = t_beg; t < t_end; ++t, ++ti) {
+            if ((ti & 1) != w) continue;
+            Tile x;
+            decode_tile(dv, rtiles, causal, t, x);
+            int32_t* out = sel + (size_t(x.bh) * dv.L + x.q0) * k;
+            if (x.ncand == 0) {
+                if (row < x.nq)
+                    for (int j = 0; j < k; ++j) out[size_t(row) * k + j] = -1;
+                continue;
+            }
+            float ts[KMAX];
+            int tj[KMAX];
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j) {
+                ts[j] = -INFINITY;
+                tj[j] = kIdNone;
+            }
+            bool stop = false;
+            for (int b = 0; b < x.nb; ++b) {
+                const int nbc = min(kBlk, x.ncand - b * kBlk);
+                if (!wait_bar_warp(bar(R_S_FULL + w), u & 1, abort, err, 25)) { stop = true; break; }
+                tc_fence_after();
+                // this row's nbc scores, 16 columns at a time (candidate ids: the same
+                // table entry for every thread, served from L1)
+                const int32_t* ids = dv.cand + x.cbeg + b * kBlk;
+                for (int c0 = 0; c0 < nbc; c0 += 16) {
+                    uint32_t sc[16];
+                    tmem_ld16(lane_addr + c0, sc);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        if (c0 + e < nbc) topk_push<KMAX>(ts, tj, __uint_as_float(sc[e]), __ldg(ids + c0 + e));
+                }
+                tc_fence_before();
+                mbar_arrive(bar(R_S_FREE + w));
+                ++u;
+            }
+            if (stop) break;
+            if (row < x.nq) {
+#pragma unroll
+                for (int j = 0; j < KMAX; ++j)
+                    if (j < k) out[size_t(row) * k + j] = (tj[j] == kIdNone) ? -1 : tj[j];
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+template <int D, int KMAX>
+cudaError_t launch_dk(const DevLayout& dv, int BH, int64_t rtiles, const void* Q, const float* Kbar, int k,
+                      int causal, int32_t* sel, cudaStream_t s) {
+    CUtensorMap tmQ;
+    if (!make_tmap(&tmQ, Q, D, int64_t(BH) * dv.L)) return cudaErrorInvalidValue;
+    const int smem = RCfg<D>::kSmem;
+    cudaError_t e = cudaFuncSetAttribute(route_tc_kernel<D, KMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(unsigned(rtiles), BH);
-    route_kernel<D, KMAX><<<grid, 256, smem, s>>>(dv, static_cast<const __nv_bfloat16*>(Q), Kbar, k,
-                                                  causal, sel);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t total = int64_t(BH) * rtiles;
+    const int grid = int(total < sms ? total : sms);
+    route_tc_kernel<D, KMAX><<<grid, kRThreads, smem, s>>>(tmQ, dv, total, rtiles, Kbar, k, causal, sel);
     return cudaGetLastError();
 }
 
 template <int D>
-cudaError_t launch_route_d(const DevLayout& dv, int BH, int64_t rtiles, const void* Q,
-                           const float* Kbar, int k, int causal, int32_t* sel, cudaStream_t s) {
-    if (k <= 4) return launch_route_dk<D, 4>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
-    if (k <= 8) return launch_route_dk<D, 8>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
-    if (k <= 16) return launch_route_dk<D, 16>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
-    return launch_route_dk<D, 32>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
+cudaError_t launch_d(const DevLayout& dv, int BH, int64_t rtiles, const void* Q, const float* Kbar, int k,
+                     int causal, int32_t* sel, cudaStream_t s) {
+    if (k <= 4) return launch_dk<D, 4>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
+    if (k <= 8) return launch_dk<D, 8>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
+    if (k <= 16) return launch_dk<D, 16>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
+    return launch_dk<D, 32>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
 }
 
 }  // namespace
 
 cudaError_t launch_route(const DevLayout& dv, int BH, int64_t rtiles, int d, const void* Q,
                          const float* Kbar, int k, int causal, int32_t* sel, cudaStream_t s) {
-    if (BH > 65535 || rtiles <= 0 || rtiles > 0x7fffffff) return cudaErrorInvalidValue;
-    if (d == 128) return launch_route_d<128>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
-    return launch_route_d<64>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
+    if (rtiles <= 0 || BH > 65535) return cudaErrorInvalidValue;
+    if (d == 128) return launch_d<128>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
+    return launch_d<64>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
 }
 
 }  // namespace moc

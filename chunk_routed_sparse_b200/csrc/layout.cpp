@@ -184,6 +184,8 @@ moc_status upload(moc_layout* lay) {
         offs.push_back(total);
         total += ((t->size() * sizeof(int32_t) + 255) / 256) * 256 + 256;
     }
+    const size_t err_off = total;  // device error word of the router (zeroed)
+    total += 256;
     std::vector<char> host(total, 0);
     for (size_t i = 0; i < tabs.size(); ++i)
         if (!tabs[i]->empty()) memcpy(host.data() + offs[i], tabs[i]->data(), tabs[i]->size() * 4);
@@ -214,6 +216,7 @@ moc_status upload(moc_layout* lay) {
     dv.rtile_off = at(9);
     dv.atile_off = at(10);
     dv.a_order = at(11);
+    dv.err = reinterpret_cast<int32_t*>(static_cast<char*>(lay->dev_block) + err_off);
     return MOC_OK;
 }
 
@@ -256,6 +259,23 @@ extern "C" moc_status moc_layout_info(const moc_layout* layout, int64_t* L, int3
     if (L) *L = layout->L;
     if (C) *C = layout->C;
     if (n_shots) *n_shots = layout->n_shots;
+    return MOC_OK;
+}
+
+extern "C" moc_status moc_layout_device_error(const moc_layout* layout, int32_t* detail,
+                                              moc_stream_t stream) {
+    if (!layout || !layout->dev_block) return MOC_ERR_INVALID_ARG;
+    int32_t h[2] = {0, 0};
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(h, layout->dv.err, sizeof h, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOC_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOC_ERR_CUDA;
+    if (detail) *detail = (h[0] != moc::ERR_NONE) ? h[1] : 0;
+    if (h[0] != moc::ERR_NONE) {
+        if (cudaMemsetAsync(layout->dv.err, 0, sizeof h, s) != cudaSuccess) return MOC_ERR_CUDA;
+        if (cudaStreamSynchronize(s) != cudaSuccess) return MOC_ERR_CUDA;
+    }
+    if (h[0] == moc::ERR_TIMEOUT) return MOC_ERR_DEVICE_TIMEOUT;
+    if (h[0] == moc::ERR_CHECK) return MOC_ERR_DEVICE_CHECK;
     return MOC_OK;
 }
 

@@ -31,6 +31,7 @@ struct DevLayout {
     const int32_t* rtile_off;    // [G+1] prefix of router tiles (kQTile queries) per group
     const int32_t* atile_off;    // [G+1] prefix of anchor items (kItemRows queries), groups in a_order
     const int32_t* a_order;      // [G] groups by descending anchor keys per tile
+    int32_t* err;                // [2] error word + detail of kernels without a workspace (router)
 };
 
 }  // namespace moc

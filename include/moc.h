@@ -193,6 +193,12 @@ moc_status moc_attention_fwd_static(const moc_layout* layout, int B, int H, int 
 moc_status moc_check_device_error(void* ws, size_t ws_bytes, int32_t* detail,
                                   moc_stream_t stream);
 
+/* Read and clear the device error word kept with a layout, where kernels that
+ * run without a workspace (the router, (2)) record a bounded wait that gave up.
+ * Synchronises the stream. Returns MOC_OK, MOC_ERR_DEVICE_TIMEOUT or
+ * MOC_ERR_DEVICE_CHECK; *detail (nullable) receives a kernel-specific code. */
+moc_status moc_layout_device_error(const moc_layout* layout, int32_t* detail, moc_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
