@@ -291,7 +291,8 @@ def run_ours(args):
                      "peak_kind": f"bf16_tflops_sustained ({peak_src})",
                      "frac_of_burst": achieved_tf / float(peaks.get("bf16_tflops", 1590.0)),
                      "traffic": traffic},
-        "hbm_kernels": hbm_fracs(stage_ms, B, H, L, lay.C, d, k, peaks),
+        "hbm_kernels": hbm_fracs(stage_ms, B, H, L, lay.C, d, k, peaks, routed_rows(lay, wl),
+                                 int((sel >= 0).sum().item()) if k > 0 else 0),
         "clocks": clk,
         "e2e": {"value": ws_ * tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                 "ms_per_step": e2e_ms,
@@ -307,14 +308,30 @@ def run_ours(args):
         torch.distributed.destroy_process_group()
 
 
-def hbm_fracs(stage_ms, B, H, L, C, d, k, peaks):
-    """Achieved GB/s of the HBM-bound kernels on their algorithmic bytes."""
+def routed_rows(lay, wl) -> int:
+    """Query rows (one head) that have at least one routing candidate."""
+    grp = lay.table(1)
+    cand_off = lay.table(5)
+    ncausal = lay.table(6)
+    rows = 0
+    for g in range(len(grp) // 2):
+        n = ncausal[g] if wl.causal else cand_off[g + 1] - cand_off[g]
+        if n > 0:
+            rows += grp[2 * g + 1] - grp[2 * g]
+    return rows
+
+
+def hbm_fracs(stage_ms, B, H, L, C, d, k, peaks, n_routed_rows, n_valid_sel):
+    """Achieved GB/s of the HBM-bound kernels on their algorithmic bytes:
+    pool reads K and writes Kbar; route reads the Q rows that have candidates
+    and writes sel; merge reads sel, the anchor partial of every row and one
+    partial per valid selection (fp32 row + lse), and writes bf16 O + lse."""
     hbm = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
     BH = B * H
     alg = {
         "pool": BH * L * 2 * d + BH * C * d * 4,
-        "route": BH * L * 2 * d + BH * L * 4 * k,
-        "merge": BH * L * ((k + 1) * (4 * d + 4) + 4 * k + 2 * d + 4),
+        "route": BH * n_routed_rows * 2 * d + BH * L * 4 * k,
+        "merge": BH * L * (4 * k + 4 * d + 4 + 2 * d + 4) + n_valid_sel * (4 * d + 4),
     }
     out = {}
     for s, b in alg.items():

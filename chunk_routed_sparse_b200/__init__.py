@@ -68,6 +68,7 @@ SIGNATURES = {
     "moc_attention_fwd_static": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _F, _P, _P, _P]),
     "moc_check_device_error": (_I, [_P, _SZ, _P, _P]),
     "moc_layout_device_error": (_I, [_P, _P, _P]),
+    "moc_selftest_bounded_wait": (_I, [_P, _P]),
 }
 
 

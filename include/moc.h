@@ -193,6 +193,14 @@ moc_status moc_attention_fwd_static(const moc_layout* layout, int B, int H, int 
 moc_status moc_check_device_error(void* ws, size_t ws_bytes, int32_t* detail,
                                   moc_stream_t stream);
 
+/* Diagnostic (the pages have no counterpart): run the bounded mbarrier wait
+ * the kernels use on a barrier nothing arrives at. After its time limit (2 s)
+ * it records ERR_TIMEOUT in dev_word[0] and a site code in dev_word[1] (device
+ * int32[2], e.g. the first bytes of an attention workspace, so that
+ * moc_check_device_error then reports MOC_ERR_DEVICE_TIMEOUT) and returns;
+ * nothing hangs or faults. Asynchronous on the stream. */
+moc_status moc_selftest_bounded_wait(int32_t* dev_word, moc_stream_t stream);
+
 /* Read and clear the device error word kept with a layout, where kernels that
  * run without a workspace (the router, (2)) record a bounded wait that gave up.
  * Synchronises the stream. Returns MOC_OK, MOC_ERR_DEVICE_TIMEOUT or

@@ -4,6 +4,7 @@ Inputs are the seeded synthetic workloads of ``moc_workloads``; the same CPU
 bytes feed the oracle and the GPU. Tolerances are in ``tests/parity.py``.
 """
 import math
+import time
 
 import numpy as np
 import pytest
@@ -228,3 +229,33 @@ def test_deterministic_repeat():
     b = moc.forward(lay, Q, K, V, 2)
     torch.cuda.synchronize()
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """A device wait that can never complete gives up after its limit, the
+    error reaches the host through the workspace error word, and the context
+    keeps working (failure detection without a GPU fault or hang)."""
+    wl = W.tiny()
+    Q, K, V = (t.cuda() for t in W.make_qkv(wl))
+    lay = moc.Layout.from_workload(wl)
+    ws = moc.workspace(lay, 1, 2, 64, 2)
+    O1, lse1, sel, _ = moc.forward(lay, Q, K, V, 2, ws=ws)
+    assert moc.check_device_error(ws) == 0
+    t0 = time.time()
+    assert moc.lib().moc_selftest_bounded_wait(moc._ptr(ws), moc._stream()) == 0
+    with pytest.raises(moc.MocError) as ei:
+        moc.check_device_error(ws)
+    assert ei.value.status == 5 and time.time() - t0 >= 1.5
+    assert moc.check_device_error(ws) == 0          # cleared
+    O2, lse2, _, _ = moc.forward(lay, Q, K, V, 2, ws=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(O1, O2) and torch.equal(lse1, lse2)
+    assert moc.check_layout_error(lay) == 0
+
+
+@pytest.mark.parametrize("anchor,causal,k", [("chunk", True, 16), ("shot", False, 4)])
+def test_ragged_scene_more_than_256_candidates(anchor, causal, k):
+    """Up to 297 candidates per group: the router's multi-block path, with
+    the own-chunk anchor and with the causal mask off."""
+    _check_full(W.ragged().replace(anchor=anchor, causal=causal), k=k, n_random=96, seed=11,
+                heads=[(0, 3), (0, 17)])
