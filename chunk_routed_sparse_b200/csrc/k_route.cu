@@ -339,7 +339,14 @@ cudaError_t launch_dk(const DevLayout& dv, int BH, int64_t rtiles, const void* Q
 template <int D>
 cudaError_t launch_d(const DevLayout& dv, int BH, int64_t rtiles, const void* Q, const float* Kbar, int k,
                      int causal, int32_t* sel, cudaStream_t s) {
-    if (k <= 4) return launch_dk<D, 4>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
+    // exact list length for small k (the insertion network costs one level per entry)
+    switch (k) {
+        case 1: return launch_dk<D, 1>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
+        case 2: return launch_dk<D, 2>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
+        case 3: return launch_dk<D, 3>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
+        case 4: return launch_dk<D, 4>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
+        default: break;
+    }
     if (k <= 8) return launch_dk<D, 8>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
     if (k <= 16) return launch_dk<D, 16>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
     return launch_dk<D, 32>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
