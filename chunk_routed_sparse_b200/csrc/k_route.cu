@@ -65,9 +65,10 @@ struct RShared {  // at oBar + 128
 
 // Insert (cs, cj) into a register list sorted by descending score (branch
 // free: one compare and four selects per entry). Candidates arrive in
-// ascending chunk id, so the strict ">" keeps an equal score behind the
-// earlier, lower id - the list is ordered by (score desc, id asc) without
-// ever comparing ids. The last entry drops out.
+// ascending chunk id (cj is the position in the ascending candidate list), so
+// the strict ">" keeps an equal score behind the earlier, lower id - the list
+// is ordered by (score desc, id asc) without ever comparing ids. The last
+// entry drops out.
 template <int KMAX>
 __device__ __forceinline__ void topk_push(float (&ts)[KMAX], int (&tj)[KMAX], float cs, int cj) {
 #pragma unroll
@@ -287,16 +288,17 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 const int nbc = min(kBlk, x.ncand - b * kBlk);
                 if (!wait_bar_warp(bar(R_S_FULL + w), u & 1, abort, err, 25)) { stop = true; break; }
                 tc_fence_after();
-                // this row's nbc scores, 16 columns at a time (candidate ids: the same
-                // table entry for every thread, served from L1)
-                const int32_t* ids = dv.cand + x.cbeg + b * kBlk;
-                for (int c0 = 0; c0 < nbc; c0 += 16) {
-                    uint32_t sc[16];
-                    tmem_ld16(lane_addr + c0, sc);
+                // this row's nbc scores, 32 columns at a time; the list carries the
+                // candidate's position in the group's list (ascending like the ids),
+                // mapped to chunk ids once the tile is done
+                for (int c0 = 0; c0 < nbc; c0 += 32) {
+                    uint32_t sc[32];
+                    tmem_ld32(lane_addr + c0, sc);
                     tmem_wait_ld();
+                    const int pos0 = b * kBlk + c0;
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        if (c0 + e < nbc) topk_push<KMAX>(ts, tj, __uint_as_float(sc[e]), __ldg(ids + c0 + e));
+                    for (int e = 0; e < 32; ++e)
+                        if (c0 + e < nbc) topk_push<KMAX>(ts, tj, __uint_as_float(sc[e]), pos0 + e);
                 }
                 tc_fence_before();
                 mbar_arrive(bar(R_S_FREE + w));
@@ -306,7 +308,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
             if (row < x.nq) {
 #pragma unroll
                 for (int j = 0; j < KMAX; ++j)
-                    if (j < k) out[size_t(row) * k + j] = (tj[j] == kIdNone) ? -1 : tj[j];
+                    if (j < k) out[size_t(row) * k + j] = (tj[j] == kIdNone) ? -1 : __ldg(dv.cand + x.cbeg + tj[j]);
             }
         }
     }
