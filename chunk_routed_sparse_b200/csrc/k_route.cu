@@ -9,23 +9,27 @@
 // spends no budget on them (they are not candidates).
 //
 // Work unit: a 128-query tile of one query group (all its queries share one
-// candidate list) times a block of <= 256 of the group's candidates. One
-// persistent CTA per SM walks a contiguous range of tiles, 320 threads:
-//   warp 8 (one lane): streams each tile's Q rows (two 64-column,
+// candidate list) times a block of the group's candidates. One persistent CTA
+// per SM walks a contiguous range of tiles with NWG selection warpgroups
+// (4 for k <= 8, else 2) and two more warps:
+//   warp 4*NWG (one lane): streams each tile's Q rows (two 64-column,
 //          128-byte-swizzled slabs) into a 2-stage ring with TMA;
-//   warp 9: owns 512 TMEM columns (one 256-column score buffer per selection
-//          warpgroup). When the (head, group, block) changes it converts the
-//          block's fp32 pooled keys into swizzled bf16 operands hi = RN(Kbar)
-//          and lo = RN(Kbar - hi) - Q is exact bf16, so the two bf16 products
-//          reproduce q . Kbar to ~2^-17 relative per term - and its lane 0
-//          issues S = Q hi^T + Q lo^T (M=128, N = block rounded up to 16,
-//          K = d, fp32 accumulation in TMEM);
-//   warps 0-3 / 4-7: two selection warpgroups taking alternate tiles; one
+//   warp 4*NWG+1: owns 512 TMEM columns (one 512/NWG-column score buffer per
+//          selection warpgroup). When the (head, group, 256-candidate operand
+//          block) changes it converts the block's fp32 pooled keys into
+//          swizzled bf16 operands hi = RN(Kbar) and lo = RN(Kbar - hi) - Q is
+//          exact bf16, so the two bf16 products reproduce q . Kbar to ~2^-17
+//          relative per term - and its lane 0 issues S = Q hi^T + Q lo^T for
+//          each 512/NWG-candidate slice of the block (M=128, N = slice rounded
+//          up to 16, K = d, fp32 accumulation in TMEM);
+//   warps 0 .. 4*NWG-1: selection warpgroups taking tiles round robin; one
 //          thread per query row (= TMEM lane) reads its scores from TMEM and
 //          keeps a sorted top-KMAX list in registers with a branch-free
 //          insertion network (candidates come in ascending id, so a strict
 //          ">" orders ties by lower chunk id), writing the first k entries
-//          (-1 padded) after the tile's last block.
+//          (-1 padded) after the tile's last slice. The network is a chain of
+//          dependent compare/select steps per row, so more warpgroups (more
+//          rows in flight per scheduler) hide its latency.
 // Tiles without candidates (caption groups, the first shot) are written as -1
 // rows by their selection warpgroup and skip the other roles. Waits are
 // bounded as in the attention kernel; a timeout is recorded in the layout's
@@ -38,9 +42,16 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kBlk = 256;  // candidates per MMA block (N <= 256)
+constexpr int kBlk = 256;  // candidates per operand block in shared memory
 constexpr int kIdNone = 0x7fffffff;
-constexpr int kRThreads = 320;
+
+template <int KMAX>
+struct RWarps {
+    static constexpr int kNwg = KMAX <= 8 ? 4 : 2;   // selection warpgroups
+    static constexpr int kSlice = 512 / kNwg;       // TMEM columns per warpgroup = candidates per MMA
+    static constexpr int kThreads = kNwg * 128 + 64;
+    static constexpr int kProducer = kNwg * 4, kIssuer = kNwg * 4 + 1;
+};
 
 template <int D>
 struct RCfg {
@@ -56,7 +67,7 @@ struct RCfg {
 };
 
 // R_S_FULL / R_S_FREE: [warpgroup]; R_KB_FREE: the MMAs that read the operand block are done
-enum { R_Q_FULL = 0, R_Q_EMPTY = 2, R_S_FULL = 4, R_S_FREE = 6, R_KB_FREE = 8, R_MMA_DONE = 9 };
+enum { R_Q_FULL = 0, R_Q_EMPTY = 2, R_S_FULL = 4, R_S_FREE = 8, R_KB_FREE = 12, R_MMA_DONE = 13 };
 
 struct RShared {  // at oBar + 128
     uint32_t tmem_base;
@@ -64,19 +75,20 @@ struct RShared {  // at oBar + 128
 };
 
 // Insert (cs, cj) into a register list sorted by descending score (branch
-// free: one compare and four selects per entry). Candidates arrive in
-// ascending chunk id (cj is the position in the ascending candidate list), so
-// the strict ">" keeps an equal score behind the earlier, lower id - the list
-// is ordered by (score desc, id asc) without ever comparing ids. The last
-// entry drops out.
+// free: per entry one compare, a max / min pair for the scores and two
+// selects for the ids; the carried score passes through a single min per
+// entry). Candidates arrive in ascending chunk id (cj is the position in the
+// ascending candidate list), so the strict ">" keeps an equal score behind the
+// earlier, lower id - the list is ordered by (score desc, id asc) without ever
+// comparing ids. The last entry drops out.
 template <int KMAX>
 __device__ __forceinline__ void topk_push(float (&ts)[KMAX], int (&tj)[KMAX], float cs, int cj) {
 #pragma unroll
     for (int x = 0; x < KMAX; ++x) {
         const bool gt = cs > ts[x];
-        const float ks = gt ? cs : ts[x];
+        const float ks = fmaxf(cs, ts[x]);
         const int kj = gt ? cj : tj[x];
-        cs = gt ? ts[x] : cs;
+        cs = fminf(cs, ts[x]);
         cj = gt ? tj[x] : cj;
         ts[x] = ks;
         tj[x] = kj;
@@ -87,6 +99,7 @@ struct Tile {
     int bh, g, q0, nq, cbeg, ncand, nb;
 };
 
+template <int SLICE>
 __device__ __forceinline__ void decode_tile(const DevLayout& dv, int64_t rtiles, int causal, int64_t t,
                                             Tile& x) {
     x.bh = int(t / rtiles);
@@ -97,7 +110,7 @@ __device__ __forceinline__ void decode_tile(const DevLayout& dv, int64_t rtiles,
     x.cbeg = dv.cand_off[x.g];
     x.ncand = (dv.grp_kind[x.g] != MOC_VIDEO) ? 0
               : causal ? dv.cand_ncausal[x.g] : dv.cand_off[x.g + 1] - x.cbeg;
-    x.nb = (x.ncand + kBlk - 1) / kBlk;
+    x.nb = (x.ncand + SLICE - 1) / SLICE;  // MMA slices
 }
 
 // Fill the hi / lo operand block (K-major, 128-byte swizzle) of candidates
@@ -135,11 +148,13 @@ __device__ __forceinline__ void build_block(const DevLayout& dv, const float* __
 }
 
 template <int D, int KMAX>
-__global__ void __launch_bounds__(kRThreads, 1)
+__global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
     route_tc_kernel(const __grid_constant__ CUtensorMap tmQ, DevLayout dv, int64_t total_tiles,
                     int64_t rtiles, const float* __restrict__ Kbar, int k, int causal,
                     int32_t* __restrict__ sel) {
     using C = RCfg<D>;
+    using WP = RWarps<KMAX>;
+    constexpr int NWG = WP::kNwg, SLICE = WP::kSlice;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -160,6 +175,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
         for (int x = 0; x < 2; ++x) {
             mbar_init(bar(R_Q_FULL + x), 1);
             mbar_init(bar(R_Q_EMPTY + x), 1);
+        }
+        for (int x = 0; x < NWG; ++x) {
             mbar_init(bar(R_S_FULL + x), 1);
             mbar_init(bar(R_S_FREE + x), 128);
         }
@@ -168,7 +185,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
         sh.abort = 0;
         fence_mbar_init();
     }
-    if (warp == 9) {
+    if (warp == WP::kIssuer) {
         tmem_alloc(smem_u32(&sh.tmem_base), 512);
         tmem_relinquish();
     }
@@ -177,14 +194,14 @@ __global__ void __launch_bounds__(kRThreads, 1)
     tc_fence_after();
     const uint32_t tmem = sh.tmem_base;
 
-    if (warp == 8) {
+    if (warp == WP::kProducer) {
         // ------------------------------------------------------------ Q producer
         if (lane == 0) {
             prefetch_tmap(&tmQ);
             uint32_t qi = 0;
             for (int64_t t = t_beg; t < t_end; ++t) {
                 Tile x;
-                decode_tile(dv, rtiles, causal, t, x);
+                decode_tile<SLICE>(dv, rtiles, causal, t, x);
                 if (x.ncand == 0) continue;
                 const int st = qi & 1;
                 if (!wait_bar(bar(R_Q_EMPTY + st), ((qi >> 1) & 1) ^ 1, abort, err, 21)) break;
@@ -200,47 +217,53 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 drain_bar(bar(R_Q_FULL + (g & 1)), (g >> 1) & 1, err, 29);
         }
         __syncwarp();
-    } else if (warp == 9) {
+    } else if (warp == WP::kIssuer) {
         // ------------------------------------------------------------ operands + MMA issue
         // The whole warp walks the units; it rebuilds the hi / lo block when the
         // (head, group, block) changes - after the MMAs that read the old block
-        // have completed - and lane 0 issues the MMAs into the score buffer of
-        // the warpgroup that owns the tile (tiles alternate between the two).
-        uint32_t qi = 0, nkb = 0, uw[2] = {0, 0};
+        // have completed - and lane 0 issues each slice's MMAs into the score
+        // buffer of the warpgroup that owns the tile (tiles go round robin).
+        uint32_t qi = 0, nkb = 0, uw[NWG];
+#pragma unroll
+        for (int i = 0; i < NWG; ++i) uw[i] = 0;
         int last_bh = -1, last_g = -1, last_b = -1, ti = 0;
         bool stop = false;
         for (int64_t t = t_beg; t < t_end && !stop; ++t, ++ti) {
             Tile x;
-            decode_tile(dv, rtiles, causal, t, x);
+            decode_tile<SLICE>(dv, rtiles, causal, t, x);
             if (x.ncand == 0) continue;
-            const int w = ti & 1;
+            const int w = ti % NWG;
             const int st = qi & 1;
             if (!wait_bar_warp(bar(R_Q_FULL + st), (qi >> 1) & 1, abort, err, 22)) break;
             for (int b = 0; b < x.nb; ++b) {
-                const int nbc = min(kBlk, x.ncand - b * kBlk);
+                const int nbc = min(SLICE, x.ncand - b * SLICE);
                 const int npad = (nbc + 15) & ~15;
-                if (x.bh != last_bh || x.g != last_g || b != last_b) {
+                const int kb = b * SLICE / kBlk;           // operand block holding this slice
+                const int roff = (b * SLICE) % kBlk;       // the slice's first row in it
+                if (x.bh != last_bh || x.g != last_g || kb != last_b) {
                     if (last_bh >= 0) {  // the previous block's MMAs are complete
                         if (lane == 0) umma_commit(bar(R_KB_FREE));
                         if (!wait_bar_warp(bar(R_KB_FREE), nkb & 1, abort, err, 23)) { stop = true; break; }
                         ++nkb;
                     }
-                    build_block<D, C::kKbSlab>(dv, Kbar, x.bh, x.cbeg, b, nbc, npad, sHi, sLo, lane);
+                    const int nbk = min(kBlk, x.ncand - kb * kBlk);
+                    build_block<D, C::kKbSlab>(dv, Kbar, x.bh, x.cbeg, kb, nbk, (nbk + 15) & ~15, sHi, sLo,
+                                               lane);
                     fence_proxy_async_smem();
                     __syncwarp();
-                    last_bh = x.bh; last_g = x.g; last_b = b;
+                    last_bh = x.bh; last_g = x.g; last_b = kb;
                 }
                 // one score buffer per warpgroup: its n-th use waits for the (n-1)-th release
                 if (!wait_bar_warp(bar(R_S_FREE + w), (uw[w] & 1) ^ 1, abort, err, 24)) { stop = true; break; }
                 tc_fence_after();
                 if (lane == 0) {
                     const uint32_t idesc = idesc_bf16_f32(128, npad, 0);
-                    const uint32_t d_s = tmem + w * 256;
+                    const uint32_t d_s = tmem + w * SLICE;
 #pragma unroll
                     for (int kk = 0; kk < 2 * (D / 16); ++kk) {  // hi then lo
                         const int kd = kk % (D / 16);
                         const uint32_t qoff = (kd >> 2) * 128 * 128 + (kd & 3) * 32;
-                        const uint32_t boff = (kd >> 2) * C::kKbSlab + (kd & 3) * 32;
+                        const uint32_t boff = (kd >> 2) * C::kKbSlab + roff * 128 + (kd & 3) * 32;
                         umma_ss(d_s, sdesc_sw128(sQ + st * C::kQBytes + qoff, 16, 1024),
                                 sdesc_sw128((kk < D / 16 ? sHi : sLo) + boff, 16, 1024), idesc, kk > 0);
                     }
@@ -260,16 +283,16 @@ __global__ void __launch_bounds__(kRThreads, 1)
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ selection (warpgroups 0, 1)
-        const int w = warp >> 2;        // this warpgroup takes tiles ti with ti % 2 == w
+        // ------------------------------------------------------------ selection warpgroups
+        const int w = warp >> 2;        // this warpgroup takes tiles ti with ti % NWG == w
         const int row = tid & 127;      // TMEM lane
-        const uint32_t lane_addr = tmem + (uint32_t((warp & 3) * 32) << 16) + w * 256;
+        const uint32_t lane_addr = tmem + (uint32_t((warp & 3) * 32) << 16) + w * SLICE;
         uint32_t u = 0;
         int ti = 0;
         for (int64_t t = t_beg; t < t_end; ++t, ++ti) {
-            if ((ti & 1) != w) continue;
+            if (ti % NWG != w) continue;
             Tile x;
-            decode_tile(dv, rtiles, causal, t, x);
+            decode_tile<SLICE>(dv, rtiles, causal, t, x);
             int32_t* out = sel + (size_t(x.bh) * dv.L + x.q0) * k;
             if (x.ncand == 0) {
                 if (row < x.nq)
@@ -285,7 +308,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
             }
             bool stop = false;
             for (int b = 0; b < x.nb; ++b) {
-                const int nbc = min(kBlk, x.ncand - b * kBlk);
+                const int nbc = min(SLICE, x.ncand - b * SLICE);
                 if (!wait_bar_warp(bar(R_S_FULL + w), u & 1, abort, err, 25)) { stop = true; break; }
                 tc_fence_after();
                 // this row's nbc scores, 32 columns at a time; the list carries the
@@ -295,7 +318,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
                     uint32_t sc[32];
                     tmem_ld32(lane_addr + c0, sc);
                     tmem_wait_ld();
-                    const int pos0 = b * kBlk + c0;
+                    const int pos0 = b * SLICE + c0;
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
                         if (c0 + e < nbc) topk_push<KMAX>(ts, tj, __uint_as_float(sc[e]), pos0 + e);
@@ -315,7 +338,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 9) {
+    if (warp == WP::kIssuer) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
@@ -334,7 +357,7 @@ cudaError_t launch_dk(const DevLayout& dv, int BH, int64_t rtiles, const void* Q
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t total = int64_t(BH) * rtiles;
     const int grid = int(total < sms ? total : sms);
-    route_tc_kernel<D, KMAX><<<grid, kRThreads, smem, s>>>(tmQ, dv, total, rtiles, Kbar, k, causal, sel);
+    route_tc_kernel<D, KMAX><<<grid, RWarps<KMAX>::kThreads, smem, s>>>(tmQ, dv, total, rtiles, Kbar, k, causal, sel);
     return cudaGetLastError();
 }
 
