@@ -59,17 +59,18 @@ struct RCfg {
     static constexpr int kQBytes = kSlabs * 128 * 128;  // one 128-row Q tile
     static constexpr int kKbSlab = kBlk * 128;          // 256 rows x 128 B
     static constexpr int kKbBytes = kSlabs * kKbSlab;   // hi (or lo) block
-    static constexpr int oQ = 0;                        // 2 stages
-    static constexpr int oHi = oQ + 2 * kQBytes;
+    static constexpr int kQStages = 2;                  // Q ring depth
+    static constexpr int oQ = 0;
+    static constexpr int oHi = oQ + kQStages * kQBytes;
     static constexpr int oLo = oHi + kKbBytes;
     static constexpr int oBar = oLo + kKbBytes;
     static constexpr int kSmem = (oBar + 256 + 1024) > 120 * 1024 ? (oBar + 256 + 1024) : 120 * 1024;
 };
 
-// R_S_FULL / R_S_FREE: [warpgroup]; R_KB_FREE: the MMAs that read the operand block are done
-enum { R_Q_FULL = 0, R_Q_EMPTY = 2, R_S_FULL = 4, R_S_FREE = 8, R_KB_FREE = 12, R_MMA_DONE = 13 };
+// R_Q_FULL / R_Q_EMPTY: [ring stage]; R_S_FULL / R_S_FREE: [warpgroup]; R_KB_FREE: the MMAs that read the operand block are done
+enum { R_Q_FULL = 0, R_Q_EMPTY = 4, R_S_FULL = 8, R_S_FREE = 12, R_KB_FREE = 16, R_MMA_DONE = 17 };
 
-struct RShared {  // at oBar + 128
+struct RShared {  // at oBar + 192 (after the barriers)
     uint32_t tmem_base;
     int abort;
 };
@@ -99,19 +100,53 @@ struct Tile {
     int bh, g, q0, nq, cbeg, ncand, nb;
 };
 
+// Walks a CTA's contiguous range of tiles (head-major, then the tiles of each
+// query group in order). A group's table entries are read when the walk
+// enters it, not per tile: each read is a dependent global load, and per-tile
+// decoding used to cost every role thousands of cycles per tile.
 template <int SLICE>
-__device__ __forceinline__ void decode_tile(const DevLayout& dv, int64_t rtiles, int causal, int64_t t,
-                                            Tile& x) {
-    x.bh = int(t / rtiles);
-    const int rt = int(t % rtiles);
-    x.g = upper_index(dv.rtile_off, dv.G + 1, rt);
-    x.q0 = dv.grp_q0[x.g] + (rt - dv.rtile_off[x.g]) * kQTile;
-    x.nq = min(kQTile, dv.grp_q1[x.g] - x.q0);
-    x.cbeg = dv.cand_off[x.g];
-    x.ncand = (dv.grp_kind[x.g] != MOC_VIDEO) ? 0
-              : causal ? dv.cand_ncausal[x.g] : dv.cand_off[x.g + 1] - x.cbeg;
-    x.nb = (x.ncand + SLICE - 1) / SLICE;  // MMA slices
-}
+struct TileWalk {
+    int bh, rt, g, rt0, rt1;  // head, tile within the head, its group and the group's tile range
+    int gq0, gq1, cbeg, ncand;
+
+    __device__ __forceinline__ void load_group(const DevLayout& dv, int causal) {
+        rt0 = dv.rtile_off[g];
+        rt1 = dv.rtile_off[g + 1];
+        gq0 = dv.grp_q0[g];
+        gq1 = dv.grp_q1[g];
+        cbeg = dv.cand_off[g];
+        ncand = (dv.grp_kind[g] != MOC_VIDEO) ? 0 : causal ? dv.cand_ncausal[g] : dv.cand_off[g + 1] - cbeg;
+    }
+    __device__ __forceinline__ void start(const DevLayout& dv, int64_t rtiles, int causal, int64_t t) {
+        bh = int(t / rtiles);
+        rt = int(t % rtiles);
+        g = upper_index(dv.rtile_off, dv.G + 1, rt);
+        load_group(dv, causal);
+    }
+    // the next tile; groups without tiles are skipped as the binary search does
+    __device__ __forceinline__ void advance(const DevLayout& dv, int64_t rtiles, int causal) {
+        if (++rt == rtiles) {
+            rt = 0;
+            ++bh;
+            g = 0;
+        } else if (rt < rt1) {
+            return;
+        }
+        while (g < dv.G - 1 && dv.rtile_off[g + 1] <= rt) ++g;
+        load_group(dv, causal);
+    }
+    __device__ __forceinline__ Tile tile() const {
+        Tile x;
+        x.bh = bh;
+        x.g = g;
+        x.q0 = gq0 + (rt - rt0) * kQTile;
+        x.nq = min(kQTile, gq1 - x.q0);
+        x.cbeg = cbeg;
+        x.ncand = ncand;
+        x.nb = (ncand + SLICE - 1) / SLICE;  // MMA slices
+        return x;
+    }
+};
 
 // Fill the hi / lo operand block (K-major, 128-byte swizzle) of candidates
 // [cbeg + b * kBlk, + nbc) of head bh; rows up to npad are zero. Run by one warp.
@@ -161,7 +196,7 @@ __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
     unsigned char* gbase = smem_raw + (base - raw);
     const uint32_t sQ = base + C::oQ, sHi = base + C::oHi, sLo = base + C::oLo;
     const uint32_t sBar = base + C::oBar;
-    RShared& sh = *reinterpret_cast<RShared*>(gbase + C::oBar + 128);
+    RShared& sh = *reinterpret_cast<RShared*>(gbase + C::oBar + 192);
     volatile int* abort = &sh.abort;
     int32_t* err = dv.err;
     auto bar = [&](int i) { return sBar + 8u * uint32_t(i); };
@@ -172,7 +207,7 @@ __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
     const int64_t t_end = total_tiles * (blockIdx.x + 1) / gridDim.x;
 
     if (tid == 0) {
-        for (int x = 0; x < 2; ++x) {
+        for (int x = 0; x < C::kQStages; ++x) {
             mbar_init(bar(R_Q_FULL + x), 1);
             mbar_init(bar(R_Q_EMPTY + x), 1);
         }
@@ -199,12 +234,13 @@ __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
         if (lane == 0) {
             prefetch_tmap(&tmQ);
             uint32_t qi = 0;
-            for (int64_t t = t_beg; t < t_end; ++t) {
-                Tile x;
-                decode_tile<SLICE>(dv, rtiles, causal, t, x);
+            TileWalk<SLICE> walk;
+            if (t_beg < t_end) walk.start(dv, rtiles, causal, t_beg);
+            for (int64_t t = t_beg; t < t_end; ++t, walk.advance(dv, rtiles, causal)) {
+                const Tile x = walk.tile();
                 if (x.ncand == 0) continue;
-                const int st = qi & 1;
-                if (!wait_bar(bar(R_Q_EMPTY + st), ((qi >> 1) & 1) ^ 1, abort, err, 21)) break;
+                const int st = qi % C::kQStages;
+                if (!wait_bar(bar(R_Q_EMPTY + st), ((qi / C::kQStages) & 1) ^ 1, abort, err, 21)) break;
                 mbar_expect_tx(bar(R_Q_FULL + st), C::kQBytes);
 #pragma unroll
                 for (int s = 0; s < C::kSlabs; ++s)
@@ -213,8 +249,8 @@ __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
                 ++qi;
             }
             // outstanding loads land before the CTA exits
-            for (uint32_t g = (qi >= 2 ? qi - 2 : 0); g < qi; ++g)
-                drain_bar(bar(R_Q_FULL + (g & 1)), (g >> 1) & 1, err, 29);
+            for (uint32_t g = (qi >= C::kQStages ? qi - C::kQStages : 0); g < qi; ++g)
+                drain_bar(bar(R_Q_FULL + g % C::kQStages), (g / C::kQStages) & 1, err, 29);
         }
         __syncwarp();
     } else if (warp == WP::kIssuer) {
@@ -228,13 +264,14 @@ __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
         for (int i = 0; i < NWG; ++i) uw[i] = 0;
         int last_bh = -1, last_g = -1, last_b = -1, ti = 0;
         bool stop = false;
-        for (int64_t t = t_beg; t < t_end && !stop; ++t, ++ti) {
-            Tile x;
-            decode_tile<SLICE>(dv, rtiles, causal, t, x);
+        TileWalk<SLICE> walk;
+        if (t_beg < t_end) walk.start(dv, rtiles, causal, t_beg);
+        for (int64_t t = t_beg; t < t_end && !stop; ++t, ++ti, walk.advance(dv, rtiles, causal)) {
+            const Tile x = walk.tile();
             if (x.ncand == 0) continue;
             const int w = ti % NWG;
-            const int st = qi & 1;
-            if (!wait_bar_warp(bar(R_Q_FULL + st), (qi >> 1) & 1, abort, err, 22)) break;
+            const int st = qi % C::kQStages;
+            if (!wait_bar_warp(bar(R_Q_FULL + st), (qi / C::kQStages) & 1, abort, err, 22)) break;
             for (int b = 0; b < x.nb; ++b) {
                 const int nbc = min(SLICE, x.ncand - b * SLICE);
                 const int npad = (nbc + 15) & ~15;
@@ -289,10 +326,11 @@ __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
         const uint32_t lane_addr = tmem + (uint32_t((warp & 3) * 32) << 16) + w * SLICE;
         uint32_t u = 0;
         int ti = 0;
-        for (int64_t t = t_beg; t < t_end; ++t, ++ti) {
+        TileWalk<SLICE> walk;
+        if (t_beg < t_end) walk.start(dv, rtiles, causal, t_beg);
+        for (int64_t t = t_beg; t < t_end; ++t, ++ti, walk.advance(dv, rtiles, causal)) {
             if (ti % NWG != w) continue;
-            Tile x;
-            decode_tile<SLICE>(dv, rtiles, causal, t, x);
+            const Tile x = walk.tile();
             int32_t* out = sel + (size_t(x.bh) * dv.L + x.q0) * k;
             if (x.ncand == 0) {
                 if (row < x.nq)
