@@ -296,13 +296,17 @@ __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
                 if (lane == 0) {
                     const uint32_t idesc = idesc_bf16_f32(128, npad, 0);
                     const uint32_t d_s = tmem + w * SLICE;
+                    // descriptors of the first K step; later steps add their byte
+                    // offset / 16 to the start-address field (no carry: < 2^14)
+                    const uint64_t dq = sdesc_sw128(sQ + st * C::kQBytes, 16, 1024);
+                    const uint64_t dhi = sdesc_sw128(sHi + roff * 128, 16, 1024);
+                    const uint64_t dlo = sdesc_sw128(sLo + roff * 128, 16, 1024);
 #pragma unroll
                     for (int kk = 0; kk < 2 * (D / 16); ++kk) {  // hi then lo
                         const int kd = kk % (D / 16);
                         const uint32_t qoff = (kd >> 2) * 128 * 128 + (kd & 3) * 32;
-                        const uint32_t boff = (kd >> 2) * C::kKbSlab + roff * 128 + (kd & 3) * 32;
-                        umma_ss(d_s, sdesc_sw128(sQ + st * C::kQBytes + qoff, 16, 1024),
-                                sdesc_sw128((kk < D / 16 ? sHi : sLo) + boff, 16, 1024), idesc, kk > 0);
+                        const uint32_t boff = (kd >> 2) * C::kKbSlab + (kd & 3) * 32;
+                        umma_ss(d_s, dq + (qoff >> 4), (kk < D / 16 ? dhi : dlo) + (boff >> 4), idesc, kk > 0);
                     }
                     umma_commit(bar(R_S_FULL + w));
                 }
