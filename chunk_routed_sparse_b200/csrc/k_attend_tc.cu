@@ -378,18 +378,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                     my_slot = 1 + (e & 31);
                 }
             }
-            // gather the warp's 32 query rows into the swizzled tile (16-byte chunks)
+            // gather the warp's 32 query rows into the swizzled tile (16-byte chunks):
+            // every load is issued before the first store, so the warp waits for
+            // one memory round trip instead of one per chunk
             constexpr int CH = D / 8;
-#pragma unroll 4
+            uint4 qv[CH];
+#pragma unroll
+            for (int i = 0; i < CH; ++i) {
+                const int tok = __shfl_sync(0xffffffffu, my_tok, (i * 32 + lane) / CH);
+                qv[i] = make_uint4(0, 0, 0, 0);
+                if (tok >= 0) qv[i] = ldg_nc16(Qb + size_t(tok) * D + ((i * 32 + lane) % CH) * 8);
+            }
+#pragma unroll
             for (int i = 0; i < CH; ++i) {
                 const int idx = i * 32 + lane;
                 const int r = (warp & 3) * 32 + idx / CH, ch = idx % CH;
-                const int tok = __shfl_sync(0xffffffffu, my_tok, r & 31);
-                uint4 v = make_uint4(0, 0, 0, 0);
-                if (tok >= 0) v = ldg_nc16(Qb + size_t(tok) * D + ch * 8);
                 const uint32_t dst = sQq + (ch >> 3) * C::kSlabBytes + r * 128 + (((ch & 7) ^ (r & 7)) << 4);
-                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(v.x), "r"(v.y),
-                             "r"(v.z), "r"(v.w) : "memory");
+                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(qv[i].x), "r"(qv[i].y),
+                             "r"(qv[i].z), "r"(qv[i].w) : "memory");
             }
             fence_proxy_async_smem();
             mbar_arrive(bar(B_Q_FULL + q));
@@ -407,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int c = 0; c < kKT / 32; ++c)
                     tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
-                tmem_wait_ld();
+                tmem_wait_ld_regs(s);
                 // keys past the range end (only in a range's last tile) -> -inf, so P = 0
                 if (nvalid < kKT) {
 #pragma unroll
@@ -442,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int c = 0; c < D / 32; ++c) {
                         uint32_t o[32];
                         tmem_ld32(o_addr + c * 32, o);
-                        tmem_wait_ld();
+                        tmem_wait_ld_regs(o);
 #pragma unroll
                         for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
                         tmem_st32(o_addr + c * 32, o);
@@ -478,24 +484,48 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++gtt;
             }
             if (stop) break;
-            // epilogue: final PV done -> O / l -> partial row, log-sum-exp
+            // epilogue: final PV done -> O / l -> partial row, log-sum-exp. Each
+            // 32-column chunk of the warp's 32 rows is staged in shared memory - in
+            // the warp's own rows of its Q tile, free once every S of the item is
+            // done and rewritten only by this warp's next gather - and written back
+            // as whole 128-byte row pieces, four rows per store instruction.
             if (!wait_bar_warp(bar(B_PV_DONE + q), (gtt - 1) & 1, abort, hdr, 14)) break;
             tc_fence_after();
             const float inv = 1.f / l;
             float* dst = (my_tok >= 0) ? o_p + ((size_t(itm.bh) * L + my_tok) * S + my_slot) * D : nullptr;
+            float* rdst[8];  // destination row of this lane in store step i: row 4i + lane / 8
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint64_t p = __shfl_sync(0xffffffffu, reinterpret_cast<uint64_t>(dst), 4 * i + (lane >> 3));
+                rdst[i] = reinterpret_cast<float*>(p);
+            }
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
                 tmem_ld32(o_addr + c * 32, o);
-                tmem_wait_ld();
-                if (dst) {
+                tmem_wait_ld_regs(o);
+                // each slab of the tile holds this warp's rows 32 (warp & 3) .. + 31 at 128 B each
+                const uint32_t stg = sQq + (c % C::kSlabs) * C::kSlabBytes + (warp & 3) * 32 * 128;
 #pragma unroll
-                    for (int x = 0; x < 32; x += 4) {
-                        float4 v = make_float4(__uint_as_float(o[x]) * inv, __uint_as_float(o[x + 1]) * inv,
-                                               __uint_as_float(o[x + 2]) * inv, __uint_as_float(o[x + 3]) * inv);
-                        *reinterpret_cast<float4*>(dst + c * 32 + x) = v;
-                    }
+                for (int x = 0; x < 8; ++x) {
+                    const uint32_t a = stg + lane * 128 + ((x ^ (lane & 7)) << 4);
+                    asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(a),
+                                 "f"(__uint_as_float(o[4 * x]) * inv), "f"(__uint_as_float(o[4 * x + 1]) * inv),
+                                 "f"(__uint_as_float(o[4 * x + 2]) * inv), "f"(__uint_as_float(o[4 * x + 3]) * inv)
+                                 : "memory");
                 }
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = 4 * i + (lane >> 3), ch = lane & 7;
+                    float4 v;
+                    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                                 : "r"(stg + r * 128 + ((ch ^ (r & 7)) << 4))
+                                 : "memory");
+                    if (rdst[i]) *reinterpret_cast<float4*>(rdst[i] + c * 32 + ch * 4) = v;
+                }
+                __syncwarp();
             }
             tc_fence_before();
             if (dst) lse_p[(size_t(itm.bh) * L + my_tok) * S + my_slot] = (m_used + log2f(l)) * 0.69314718055994531f;

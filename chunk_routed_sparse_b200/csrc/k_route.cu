@@ -359,7 +359,7 @@ __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
                 for (int c0 = 0; c0 < nbc; c0 += 32) {
                     uint32_t sc[32];
                     tmem_ld32(lane_addr + c0, sc);
-                    tmem_wait_ld();
+                    tmem_wait_ld_regs(sc);
                     const int pos0 = b * SLICE + c0;
 #pragma unroll
                     for (int e = 0; e < 32; ++e)

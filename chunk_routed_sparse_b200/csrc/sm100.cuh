@@ -103,6 +103,16 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
                  : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// tcgen05.wait::ld, then an empty asm that reads and rewrites each register a
+// tcgen05.ld filled: the values are undefined until the wait, and without this
+// tie nothing stops the compiler from scheduling arithmetic on them (a pure
+// function of the asm outputs) above the wait.
+template <int N>
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[N]) {
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // 32 consecutive 32-bit columns of this thread's TMEM lane (warp w of a
