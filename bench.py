@@ -234,23 +234,26 @@ def run_ours(args):
                 for j, s in enumerate(STAGES)}
     moc.check_device_error(ws)
 
-    # end to end through the public API: pinned host inputs -> device -> result back
+    # end to end through the C ABI's host-buffer call (moc_forward_host): pinned host
+    # Q, K, V in, host O back; inside, chunks of heads are uploaded, computed and
+    # downloaded on three streams so that the copies overlap the kernels
     Oh = torch.empty_like(Qh).pin_memory()
+    devbuf = torch.empty(moc.forward_host_device_bytes(lay, B, H, d, k), dtype=torch.uint8, device=dev)
+    moc.forward_host(lay, Qh, Kh, Vh, k, causal=wl.causal, scale=scale, dev=devbuf, out=Oh,
+                     want_lse=False)  # untimed first call
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2e_steps = max(1, min(args.steps, 5))
     barrier()
     torch.cuda.synchronize()
     e0.record(stream)
     for _ in range(e2e_steps):
-        Q.copy_(Qh, non_blocking=True)
-        K.copy_(Kh, non_blocking=True)
-        V.copy_(Vh, non_blocking=True)
-        step()
-        Oh.copy_(O, non_blocking=True)
+        moc.forward_host(lay, Qh, Kh, Vh, k, causal=wl.causal, scale=scale, dev=devbuf, out=Oh,
+                         want_lse=False)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    del devbuf
 
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
 
@@ -296,6 +299,7 @@ def run_ours(args):
         "clocks": clk,
         "e2e": {"value": ws_ * tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                 "ms_per_step": e2e_ms,
+                "path": "moc_forward_host: host buffers, 8 chunks of heads, copies overlapped",
                 "h2d_bytes_per_step": 3 * Q.numel() * 2, "d2h_bytes_per_step": O.numel() * 2},
         "gpu_launches": args.steps * sum(LAUNCHES_PER_STEP.values()),
     }

@@ -69,6 +69,8 @@ SIGNATURES = {
     "moc_check_device_error": (_I, [_P, _SZ, _P, _P]),
     "moc_layout_device_error": (_I, [_P, _P, _P]),
     "moc_selftest_bounded_wait": (_I, [_P, _P]),
+    "moc_forward_host": (_I, [_P, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _P, _P, _P, _SZ, _I, _P]),
+    "moc_forward_host_device_bytes": (_SZ, [_P, _I, _I, _I, _I, _I]),
 }
 
 
@@ -240,6 +242,41 @@ def forward(layout: Layout, Q, K, V, k: int, causal: bool = True, scale=None, ws
         torch.empty(Q.shape[0], Q.shape[1], Q.shape[2], 0, dtype=torch.int32, device=Q.device)
     O, lse = attention_fwd(layout, Q, K, V, sel, k, scale=scale, ws=ws)
     return O, lse, sel, kbar
+
+
+def forward_host_device_bytes(layout: Layout, B: int, H: int, d: int, k: int, heads_per_chunk: int = 0) -> int:
+    return int(lib().moc_forward_host_device_bytes(layout.handle, B, H, d, k, heads_per_chunk))
+
+
+def forward_host(layout: Layout, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, k: int,
+                 causal: bool = True, scale=None, heads_per_chunk: int = 0,
+                 dev: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                 want_lse: bool = True, want_sel: bool = False):
+    """Whole forward pass on host tensors (moc_forward_host): Q, K, V are CPU bf16
+    [B, H, L, d] (pinned for overlap); returns CPU (O, lse or None, sel or None)
+    once complete. ``dev`` is the device scratch (allocated here if None)."""
+    if Q.dim() != 4:
+        raise ValueError("expected [B, H, L, d] tensors")
+    B, H, L, d = tuple(Q.shape)
+    for t in (Q, K, V):
+        if t.device.type != "cpu" or not t.is_contiguous() or t.dtype != torch.bfloat16:
+            raise ValueError("Q, K, V must be contiguous bf16 CPU tensors")
+        if tuple(t.shape) != (B, H, L, d):
+            raise ValueError("Q, K, V shapes differ")
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if dev is None:
+        n = forward_host_device_bytes(layout, B, H, d, k, heads_per_chunk)
+        if n == 0:
+            raise ValueError("invalid problem for moc_forward_host")
+        dev = torch.empty(n, dtype=torch.uint8, device=torch.cuda.current_device())
+    O = out if out is not None else torch.empty_like(Q)
+    lse = torch.empty(B, H, L, dtype=torch.float32) if want_lse else None
+    sel = torch.empty(B, H, L, k, dtype=torch.int32) if (want_sel and k > 0) else None
+    _check(lib().moc_forward_host(layout.handle, B, H, d, k, 1 if causal else 0, float(scale),
+                                  _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse), _ptr(sel),
+                                  _ptr(dev), dev.numel(), heads_per_chunk, _stream()),
+           "moc_forward_host")
+    return O, lse, sel
 
 
 def check_layout_error(layout: Layout) -> int:

@@ -147,10 +147,10 @@ moc_status moc_build_qlists(const moc_layout* layout, int B, int H, int k, const
                             void* ws, size_t ws_bytes, moc_stream_t stream);
 
 /* (4) Chunk-major attention over the work items (Summary §3.1 attention over
- * Omega(q)): per 128-query tile of a query group, attention over the group's
- * anchor key ranges (partial slot 0); per 128 entries of a chunk's query list,
- * attention of the gathered query rows over that chunk (slot 1 + position in
- * sel). Each partial is the normalised softmax output and its log-sum-exp of
+ * Omega(q)): per 256 consecutive queries of a query group, attention over the
+ * group's anchor key ranges (partial slot 0); per 256 entries of a chunk's
+ * query list, attention of the gathered query rows over that chunk (slot 1 +
+ * position in sel). Each partial is the normalised softmax output and its log-sum-exp of
  * the raw scaled scores. softmax_scale is normally 1/sqrt(d). Needs the
  * workspace filled by (3) for the same sel. */
 moc_status moc_attend_partials(const moc_layout* layout, int B, int H, int d, const void* Q,
@@ -185,6 +185,32 @@ moc_status moc_attention_fwd(const moc_layout* layout, int B, int H, int d, cons
 moc_status moc_attention_fwd_static(const moc_layout* layout, int B, int H, int d, const void* Q,
                                     const void* K, const void* V, const int32_t* sel, int k,
                                     float softmax_scale, void* O, float* lse, moc_stream_t stream);
+
+/* Whole forward pass on HOST buffers: (1) pooling, (2) routing (when k > 0)
+ * and (3)-(5) for every (b, h) slice, the end-to-end call for inputs that live
+ * in host memory. Q, K, V: host bf16 [B][H][L][d] (page-locked memory lets the
+ * copies run concurrently with the kernels); O: host bf16 [B][H][L][d]; lse
+ * (nullable): host fp32 [B][H][L]; sel (nullable): host int32 [B][H][L][k].
+ * The slices are processed in chunks of heads_per_chunk consecutive (b, h)
+ * slices (<= 0: eight chunks): chunk c+1's inputs are copied in while chunk c
+ * is computed on `stream` and chunk c-1's outputs are copied out, each of the
+ * three on its own stream. Every stage is independent per (b, h) (Summary
+ * §3.1; "計算效率": head-independent operations), so results are bitwise those
+ * of the device calls on the whole tensors. dev: device scratch of
+ * moc_forward_host_device_bytes() bytes, 256-byte aligned (two input and two
+ * output stages, pooled keys and the attention workspace of one chunk);
+ * nothing is allocated on the device. Work already queued on `stream` runs
+ * first; the call synchronises and returns when the host outputs are
+ * complete, reporting a device error word as moc_check_device_error and
+ * moc_layout_device_error do. */
+moc_status moc_forward_host(const moc_layout* layout, int B, int H, int d, int k, int causal,
+                            float softmax_scale, const void* Q, const void* K, const void* V,
+                            void* O, float* lse, int32_t* sel, void* dev, size_t dev_bytes,
+                            int heads_per_chunk, moc_stream_t stream);
+
+/* Bytes of device scratch moc_forward_host needs (0 on invalid arguments). */
+size_t moc_forward_host_device_bytes(const moc_layout* layout, int B, int H, int d, int k,
+                                     int heads_per_chunk);
 
 /* Read and clear the device error word the kernels set when a bounded wait
  * gives up or a consistency check fails. Synchronises the stream. Returns

@@ -110,6 +110,28 @@ def test_compute_calls_reject_host_only_layout():
     assert lib.moc_route(lay.handle, 1, 2, 64, p, p, 2, 1, p, None) == 1
     assert lib.moc_attention_fwd(lay.handle, 1, 2, 64, p, p, p, p, 2, 0.125, p, None, p,
                                  1 << 30, None) == 1
+    assert lib.moc_forward_host(lay.handle, 1, 2, 64, 2, 1, 0.125, p, p, p, p, None, None, p,
+                                1 << 30, 0, None) == 1
+
+
+def test_host_pipeline_device_bytes():
+    """Scratch of the host-buffer pipeline: two input stages (Q, K, V) and two
+    output stages (O, lse, sel) of one chunk, its pooled keys and its attention
+    workspace - it shrinks with the chunk and needs no GPU to size."""
+    wl = W.eight()
+    lay = _host_layout(wl)
+    lib = moc.lib()
+    per_head = wl.L * 128 * 2
+    n8 = lib.moc_forward_host_device_bytes(lay.handle, 1, 24, 128, 3, 0)    # default: 8 chunks of 3
+    n3 = lib.moc_forward_host_device_bytes(lay.handle, 1, 24, 128, 3, 3)
+    n24 = lib.moc_forward_host_device_bytes(lay.handle, 1, 24, 128, 3, 24)
+    assert n8 == n3
+    ws3 = lay.workspace_bytes(1, 3, 128, 3)
+    assert n3 >= 3 * (2 * 3 + 2) * per_head + ws3
+    assert n3 < n24 and n24 >= lay.workspace_bytes(1, 24, 128, 3) + 8 * 24 * per_head
+    assert lib.moc_forward_host_device_bytes(lay.handle, 1, 24, 128, 3, 100) == n24  # clamped to B*H
+    assert lib.moc_forward_host_device_bytes(lay.handle, 1, 24, 96, 3, 0) == 0
+    assert lib.moc_forward_host_device_bytes(None, 1, 24, 128, 3, 0) == 0
 
 
 def test_workspace_size_query():
