@@ -48,8 +48,10 @@ def load_peaks():
     return dict(PEAKS_FALLBACK), "fallback"
 
 
-def workload(name: str, k):
+def workload(name: str, k, heads=None):
     wl = W.CONFIGS[name]()
+    if heads is not None:  # fewer heads of the same scene (profiling captures)
+        wl = wl.replace(H=heads)
     return wl.with_k(k) if k is not None else wl
 
 
@@ -175,7 +177,7 @@ def run_ours(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    wl = scene_for_rank(workload(args.config, args.k), rank)
+    wl = scene_for_rank(workload(args.config, args.k, args.heads), rank)
     B, H, L, d, k = wl.B, wl.H, wl.L, wl.d, wl.k
     Qh, Kh, Vh = W.make_qkv(wl)
     Qh, Kh, Vh = Qh.pin_memory(), Kh.pin_memory(), Vh.pin_memory()
@@ -303,6 +305,9 @@ def run_ours(args):
                 "h2d_bytes_per_step": 3 * Q.numel() * 2, "d2h_bytes_per_step": O.numel() * 2},
         "gpu_launches": args.steps * sum(LAUNCHES_PER_STEP.values()),
     }
+    if ws_ == 1 and not args.no_dense_compare and wl.name == "eight":
+        line["dense_compare"] = dense_compare(moc, wl, Q, K, V, O, lse, stream, pairs,
+                                              stage_ms, ms_per_step, peak_tf)
     if rank == 0 and ws_ == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, Qh, Kh, Vh, budget_s=args.cpu_budget)
     if rank == 0:
@@ -310,6 +315,60 @@ def run_ours(args):
     if ws_ > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
+
+
+def dense_compare(moc, wl, Q, K, V, O, lse, stream, moc_pairs, stage_ms, moc_step_ms, peak_tf):
+    """The same attention kernel on two anchor-only layouts of the scene's length
+    (k = 0, so no routing and one partial per row):
+      dense - one caption segment and one shot holding every frame, so every
+              query attends every key (L^2 pairs per head);
+      flop_matched - seven shots of 6 x 28,405 + 10,082 tokens, block-diagonal
+              dense attention with the MoC scene's kept-pair count (within 0.02 %),
+              which separates the pruning gain from the cost of routing, query
+              lists, gathered tiles and the merge.
+    Pool -> attention (query lists, attend, merge) is timed with CUDA events over
+    3 runs after 2 warm-up runs, on the resident Q, K, V."""
+    import moc_workloads as Wm
+    L, d, H = wl.L, wl.d, wl.H
+    n_cap = sum(sg.length for sg in wl.segments if sg.kind == Wm.CAPTION)
+    scenes = {
+        "dense": [Wm.Segment(n_cap, Wm.CAPTION, -1, -1)]
+                 + [Wm.Segment(1500, Wm.VIDEO, 0, f) for f in range((L - n_cap) // 1500)],
+        "flop_matched": [Wm.Segment(28405, Wm.VIDEO, s_, 0) for s_ in range(6)]
+                        + [Wm.Segment(L - 6 * 28405, Wm.VIDEO, 6, 0)],
+    }
+    out = {}
+    for name, segs in scenes.items():
+        assert sum(sg.length for sg in segs) == L
+        w2 = Wm.custom(name, 1, H, d, segs, anchor="shot", causal=True, k=0)
+        lay = moc.Layout.from_workload(w2, device=Q.device.index)
+        ws = moc.workspace(lay, 1, H, d, 0, Q.device)
+        kbar = torch.empty(1, H, lay.C, d, dtype=torch.float32, device=Q.device)
+        # dense: every query sees every key; block-diagonal: every query its own block
+        pairs = H * L * L if name == "dense" else H * sum(sg.length ** 2 for sg in segs)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        att, tot = [], []
+        for it in range(5):
+            ev[0].record(stream)
+            moc.pool_keys(lay, K, out=kbar)
+            ev[1].record(stream)
+            moc.attention_fwd(lay, Q, K, V, None, 0, ws=ws, O=O, lse=lse)
+            ev[2].record(stream)
+            torch.cuda.synchronize()
+            if it >= 2:
+                tot.append(ev[0].elapsed_time(ev[2]))
+                att.append(ev[1].elapsed_time(ev[2]))
+        moc.check_device_error(ws)
+        a, t = statistics.mean(att), statistics.mean(tot)
+        out[name] = {"pairs": pairs, "attention_ms": a, "step_ms": t,
+                     "tflops": 4.0 * d * pairs / (a / 1e3) / 1e12,
+                     "frac_sustained": 4.0 * d * pairs / (a / 1e3) / 1e12 / peak_tf}
+        del ws
+    moc_attention_ms = stage_ms["qlist"] + stage_ms["attend"] + stage_ms["merge"]
+    out["moc_pairs"] = moc_pairs
+    out["moc_step_speedup_vs_dense"] = out["dense"]["step_ms"] / moc_step_ms
+    out["moc_attention_vs_flop_matched"] = moc_attention_ms / out["flop_matched"]["attention_ms"]
+    return out
 
 
 def routed_rows(lay, wl) -> int:
@@ -379,7 +438,7 @@ def run_reference(args):
     ws_, rank, _ = dist_env()
     if rank != 0:
         return
-    wl = workload(args.config, args.k)
+    wl = workload(args.config, args.k, args.heads)
     Qh, Kh, Vh = W.make_qkv(wl, heads=[(0, 0)])
     import oracle
     w1 = wl.replace(B=1, H=1)
@@ -427,8 +486,12 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="eight", choices=sorted(W.CONFIGS))
     ap.add_argument("--k", type=int, default=None)
+    ap.add_argument("--heads", type=int, default=None,
+                    help="run the scene with this many heads instead (small profiling captures)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense-compare", action="store_true",
+                    help="skip the dense and FLOP-matched block-diagonal runs of the attention kernel")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
