@@ -301,7 +301,7 @@ def run_ours(args):
         "clocks": clk,
         "e2e": {"value": ws_ * tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                 "ms_per_step": e2e_ms,
-                "path": "moc_forward_host: host buffers, 8 chunks of heads, copies overlapped",
+                "path": "moc_forward_host: host buffers, 12 chunks of heads, copies overlapped",
                 "h2d_bytes_per_step": 3 * Q.numel() * 2, "d2h_bytes_per_step": O.numel() * 2},
         "gpu_launches": args.steps * sum(LAUNCHES_PER_STEP.values()),
     }

@@ -14,7 +14,10 @@
 namespace moc {
 namespace {
 
-template <int D>
+// MAXS > 0: at most MAXS slots, every valid slot's partial loaded at once (one
+// memory round trip for sel and the log-sum-exps, one for the partials);
+// MAXS == 0: any slot count, partials loaded slot by slot.
+template <int D, int MAXS>
 __global__ void __launch_bounds__(256) merge_kernel(int64_t rows, int L, int k,
                                                     const int32_t* __restrict__ sel,
                                                     const float* __restrict__ lse_p,
@@ -26,12 +29,16 @@ __global__ void __launch_bounds__(256) merge_kernel(int64_t rows, int L, int k,
     const int S = k + 1;
     for (int64_t row = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; row < rows;
          row += (int64_t(gridDim.x) * blockDim.x) >> 5) {
-        bool valid = false;
+        // sel and the slot log-sum-exps in one round trip (an invalid slot's lse is
+        // never used: it may not have been written)
+        int32_t sj = 0;
         float l = -INFINITY;
         if (lane < S) {
-            valid = (lane == 0) || (sel[row * k + lane - 1] >= 0);
-            if (valid) l = lse_p[row * S + lane];
+            if (lane > 0) sj = __ldg(sel + row * k + lane - 1);
+            l = __ldg(lse_p + row * S + lane);
         }
+        const bool valid = lane < S && (lane == 0 || sj >= 0);
+        if (!valid) l = -INFINITY;
         float m = l;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -44,15 +51,42 @@ __global__ void __launch_bounds__(256) merge_kernel(int64_t rows, int L, int k,
 #pragma unroll
         for (int x = 0; x < PER; ++x) acc[x] = 0.f;
         const float* op = o_p + size_t(row) * S * D + lane * PER;
-        for (unsigned mm = vmask; mm; mm &= mm - 1) {
-            const int j = __ffs(mm) - 1;
-            const float wj = __shfl_sync(0xffffffffu, w, j) / z;
-            if (PER == 4) {
-                const float4 v = *reinterpret_cast<const float4*>(op + size_t(j) * D);
-                acc[0] += wj * v.x; acc[1] += wj * v.y; acc[2] += wj * v.z; acc[3] += wj * v.w;
-            } else {
-                const float2 v = *reinterpret_cast<const float2*>(op + size_t(j) * D);
-                acc[0] += wj * v.x; acc[1] += wj * v.y;
+        if (MAXS > 0) {
+            float v[MAXS > 0 ? MAXS : 1][PER];
+#pragma unroll
+            for (int j = 0; j < MAXS; ++j) {
+#pragma unroll
+                for (int x = 0; x < PER; ++x) v[j][x] = 0.f;
+                if ((vmask >> j) & 1u) {
+                    if (PER == 4) {
+                        const float4 t = __ldg(reinterpret_cast<const float4*>(op + size_t(j) * D));
+                        v[j][0] = t.x; v[j][1] = t.y; v[j][2] = t.z; v[j][3] = t.w;
+                    } else {
+                        const float2 t = __ldg(reinterpret_cast<const float2*>(op + size_t(j) * D));
+                        v[j][0] = t.x; v[j][1] = t.y;
+                    }
+                }
+            }
+            // fixed slot order, as in the general path
+#pragma unroll
+            for (int j = 0; j < MAXS; ++j) {
+                const float wj = __shfl_sync(0xffffffffu, w, j) / z;
+                if ((vmask >> j) & 1u) {
+#pragma unroll
+                    for (int x = 0; x < PER; ++x) acc[x] += wj * v[j][x];
+                }
+            }
+        } else {
+            for (unsigned mm = vmask; mm; mm &= mm - 1) {
+                const int j = __ffs(mm) - 1;
+                const float wj = __shfl_sync(0xffffffffu, w, j) / z;
+                if (PER == 4) {
+                    const float4 t = __ldg(reinterpret_cast<const float4*>(op + size_t(j) * D));
+                    acc[0] += wj * t.x; acc[1] += wj * t.y; acc[2] += wj * t.z; acc[3] += wj * t.w;
+                } else {
+                    const float2 t = __ldg(reinterpret_cast<const float2*>(op + size_t(j) * D));
+                    acc[0] += wj * t.x; acc[1] += wj * t.y;
+                }
             }
         }
         __nv_bfloat16* orow = O + size_t(row) * D + lane * PER;
@@ -78,12 +112,16 @@ cudaError_t launch_merge(int BH, int L, int d, int k, const int32_t* sel, void* 
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t want = (rows + 7) / 8;
     const int grid = int(want < int64_t(sms) * 16 ? want : int64_t(sms) * 16);
-    if (d == 128)
-        merge_kernel<128><<<grid, 256, 0, s>>>(rows, L, k, sel, lse_p, o_p,
-                                               static_cast<__nv_bfloat16*>(O), lse);
-    else
-        merge_kernel<64><<<grid, 256, 0, s>>>(rows, L, k, sel, lse_p, o_p,
-                                              static_cast<__nv_bfloat16*>(O), lse);
+    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(O);
+    if (d == 128) {
+        if (k + 1 <= 4) merge_kernel<128, 4><<<grid, 256, 0, s>>>(rows, L, k, sel, lse_p, o_p, o, lse);
+        else if (k + 1 <= 8) merge_kernel<128, 8><<<grid, 256, 0, s>>>(rows, L, k, sel, lse_p, o_p, o, lse);
+        else merge_kernel<128, 0><<<grid, 256, 0, s>>>(rows, L, k, sel, lse_p, o_p, o, lse);
+    } else {
+        if (k + 1 <= 4) merge_kernel<64, 4><<<grid, 256, 0, s>>>(rows, L, k, sel, lse_p, o_p, o, lse);
+        else if (k + 1 <= 8) merge_kernel<64, 8><<<grid, 256, 0, s>>>(rows, L, k, sel, lse_p, o_p, o, lse);
+        else merge_kernel<64, 0><<<grid, 256, 0, s>>>(rows, L, k, sel, lse_p, o_p, o, lse);
+    }
     return cudaGetLastError();
 }
 

@@ -122,10 +122,11 @@ def test_host_pipeline_device_bytes():
     lay = _host_layout(wl)
     lib = moc.lib()
     per_head = wl.L * 128 * 2
-    n8 = lib.moc_forward_host_device_bytes(lay.handle, 1, 24, 128, 3, 0)    # default: 8 chunks of 3
+    n0 = lib.moc_forward_host_device_bytes(lay.handle, 1, 24, 128, 3, 0)    # default: 12 chunks of 2
+    n2 = lib.moc_forward_host_device_bytes(lay.handle, 1, 24, 128, 3, 2)
     n3 = lib.moc_forward_host_device_bytes(lay.handle, 1, 24, 128, 3, 3)
     n24 = lib.moc_forward_host_device_bytes(lay.handle, 1, 24, 128, 3, 24)
-    assert n8 == n3
+    assert n0 == n2 < n3
     ws3 = lay.workspace_bytes(1, 3, 128, 3)
     assert n3 >= 3 * (2 * 3 + 2) * per_head + ws3
     assert n3 < n24 and n24 >= lay.workspace_bytes(1, 24, 128, 3) + 8 * 24 * per_head
