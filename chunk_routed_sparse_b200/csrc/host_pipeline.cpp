@@ -12,6 +12,7 @@
 // stages. Events order the reuse of each stage. Nothing is allocated on the
 // device: the caller passes one buffer of moc_forward_host_device_bytes().
 #include <cstring>
+#include <vector>
 
 #include "moc_internal.h"
 
@@ -115,7 +116,21 @@ extern "C" moc_status moc_forward_host(const moc_layout* lay, int B, int H, int 
     char* base = static_cast<char*>(dev);
     const size_t L = size_t(lay->L);
     const size_t row_bytes = L * size_t(d) * 2;  // one (b, h) slice of Q, K, V or O
-    const int nch = (BH + p.hc - 1) / p.hc;
+    // chunk boundaries: the first and the last chunk are half size, so that the
+    // pipeline fills (first upload) and drains (last download) sooner
+    std::vector<int> bounds{0};
+    {
+        const int half = p.hc > 1 ? p.hc / 2 : 1;
+        int h = half < BH ? half : BH;
+        bounds.push_back(h);
+        const int last = (BH - h) < half ? (BH - h) : half;
+        while (h < BH - last) {
+            h += (BH - last - h) < p.hc ? (BH - last - h) : p.hc;
+            bounds.push_back(h);
+        }
+        if (last > 0) bounds.push_back(BH);
+    }
+    const int nch = int(bounds.size()) - 1;
     auto ck = [](cudaError_t e) { return e == cudaSuccess; };
 
     // the copies start after whatever the caller queued on its stream before this call
@@ -125,7 +140,7 @@ extern "C" moc_status moc_forward_host(const moc_layout* lay, int B, int H, int 
     const size_t ws_bytes = p.ws;
     for (int c = 0; c < nch; ++c) {
         const int s = c & 1;
-        const int h0 = c * p.hc, nh = (h0 + p.hc <= BH) ? p.hc : BH - h0;
+        const int h0 = bounds[c], nh = bounds[c + 1] - bounds[c];
         char* in = base + p.off_in[s];
         char* dq = in;
         char* dk = in + p.qkv;

@@ -192,7 +192,8 @@ moc_status moc_attention_fwd_static(const moc_layout* layout, int B, int H, int 
  * copies run concurrently with the kernels); O: host bf16 [B][H][L][d]; lse
  * (nullable): host fp32 [B][H][L]; sel (nullable): host int32 [B][H][L][k].
  * The slices are processed in chunks of heads_per_chunk consecutive (b, h)
- * slices (<= 0: twelve chunks): chunk c+1's inputs are copied in while chunk c
+ * slices (<= 0: B*H/12 rounded up; the first and the last chunk are half
+ * that): chunk c+1's inputs are copied in while chunk c
  * is computed on `stream` and chunk c-1's outputs are copied out, each of the
  * three on its own stream. Every stage is independent per (b, h) (Summary
  * §3.1; "計算效率": head-independent operations), so results are bitwise those
