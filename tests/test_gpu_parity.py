@@ -137,6 +137,22 @@ def test_stress_scene_two_heads():
     _check_full(W.stress(), n_random=64, seed=5, heads=[(0, 0), (1, 23)])
 
 
+@pytest.mark.parametrize("name,k,pairs", [("eight", 2, 4_707_082_144), ("stress", 8, 12_888_328_576)])
+def test_kept_pairs_match_closed_form(name, k, pairs):
+    """The number of kept (query, key) pairs per (b, h) depends only on the
+    layout and k (every query keeps min(k, |candidates|) chunks), so the GPU
+    routing of every head - data-carrying or all-zero (ties to the lowest ids)
+    - must give the closed-form count exactly; eight-shot k=2 and stress k=8."""
+    wl = W.CONFIGS[name]().with_k(k)
+    heads = [(0, 0), (wl.B - 1, wl.H - 1)]
+    Q, K, V = W.make_qkv(wl, heads=heads)
+    lay, O, lse, sel, kbar = _run(wl, Q, K, V)
+    orc = oracle.Layout(wl)
+    for b in range(wl.B):
+        for h in (0, wl.H // 2, wl.H - 1):
+            assert oracle.kept_pairs(wl, sel[b, h], orc) == pairs, (b, h)
+
+
 def test_empty_batch_is_a_noop():
     wl = W.tiny()
     lay = moc.Layout.from_workload(wl)
