@@ -46,12 +46,13 @@ def poisson_thresholds(lam: float, m_max: int) -> List[int]:
     """thr[i] = floor(F(i) * 2^32) for the Poisson(lam) distribution function
     F(i) = sum_{j <= i} e^-lam lam^j / j!, accumulated in double from
     p_0 = exp(-lam), p_j = p_{j-1} * lam / j; m = #{i < m_max : thr[i] <= w}."""
+    lam = float(np.float32(lam))  # the rates are single-precision arguments of the call
     thr = []
-    p = math.exp(-float(lam))
+    p = math.exp(-lam)
     cdf = p
     for i in range(m_max):
         if i > 0:
-            p = p * float(lam) / float(i)
+            p = p * lam / float(i)
             cdf = cdf + p
         thr.append(min(int(math.floor(cdf * 4294967296.0)), 1 << 32))
     return thr
