@@ -71,6 +71,7 @@ SIGNATURES = {
     "moc_selftest_bounded_wait": (_I, [_P, _P]),
     "moc_forward_host": (_I, [_P, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _P, _P, _P, _SZ, _I, _P]),
     "moc_forward_host_device_bytes": (_SZ, [_P, _I, _I, _I, _I, _I]),
+    "moc_route_perturb": (_I, [_P, _I, _I, _I, _I, _P, _P, _F, _F, _I, _P, _P]),
 }
 
 
@@ -185,6 +186,25 @@ def route(layout: Layout, Q: torch.Tensor, kbar: torch.Tensor, k: int, causal: b
         out = torch.empty(B, H, L, k, dtype=torch.int32, device=Q.device)
     _check(lib().moc_route(layout.handle, B, H, d, _ptr(Q), _ptr(kbar), k, int(bool(causal)),
                            _ptr(out), _stream()), "moc_route")
+    return out
+
+
+def route_perturb(layout: Layout, sel: Optional[torch.Tensor], rnd: torch.Tensor, k: int, p_max: float,
+                  lam: float, m_max: int, causal: bool = True, B: Optional[int] = None,
+                  H: Optional[int] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Context drop-off / drop-in (moc_route_perturb): sel int32 [B, H, L, k] from
+    route() (None when k == 0), rnd uint32-valued int32 [B, H, L, 2 + k + m_max]
+    of random words; returns int32 [B, H, L, k + m_max]."""
+    B = rnd.shape[0] if B is None else B
+    H = rnd.shape[1] if H is None else H
+    L = rnd.shape[2]
+    if rnd.shape[3] != 2 + k + m_max or not rnd.is_cuda or rnd.dtype not in (torch.int32, torch.uint32):
+        raise ValueError("rnd must be a CUDA int32/uint32 tensor [B, H, L, 2 + k + m_max]")
+    if out is None:
+        out = torch.empty(B, H, L, k + m_max, dtype=torch.int32, device=rnd.device)
+    _check(lib().moc_route_perturb(layout.handle, B, H, k, 1 if causal else 0,
+                                   _ptr(sel) if k > 0 else None, _ptr(rnd), float(p_max), float(lam),
+                                   m_max, _ptr(out), _stream()), "moc_route_perturb")
     return out
 
 

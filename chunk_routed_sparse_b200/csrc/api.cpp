@@ -1,6 +1,7 @@
 // C-ABI entry points: argument validation, workspace carve-up and kernel
 // launches. Every compute call is asynchronous on the caller's stream and
 // allocates nothing.
+#include <cmath>
 #include <cstring>
 
 #include "moc_internal.h"
@@ -89,6 +90,35 @@ extern "C" moc_status moc_route(const moc_layout* lay, int B, int H, int d, cons
         return MOC_ERR_INVALID_ARG;
     return cuda_status(moc::launch_route(lay->dv, B * H, lay->total_rtiles, d, Q, Kbar, k,
                                          causal ? 1 : 0, sel, (cudaStream_t)stream));
+}
+
+extern "C" moc_status moc_route_perturb(const moc_layout* lay, int B, int H, int k, int causal,
+                                        const int32_t* sel, const uint32_t* rnd, float p_max,
+                                        float lambda, int m_max, int32_t* sel_out, moc_stream_t stream) {
+    moc_status st = check_common(lay, B, H, 128, k);
+    if (st != MOC_OK) return st;
+    if (m_max < 0 || k + m_max > moc::kMaxK || k + m_max == 0) return MOC_ERR_INVALID_ARG;
+    if (!(p_max >= 0.0f && p_max <= 1.0f) || !(lambda >= 0.0f) || !std::isfinite(lambda))
+        return MOC_ERR_INVALID_ARG;
+    if (B * H == 0) return MOC_OK;
+    if (int64_t(B) * H * lay->L * (2 + k + m_max) >= (int64_t(1) << 31)) return MOC_ERR_UNSUPPORTED;
+    if ((k > 0 && (!sel || (reinterpret_cast<uintptr_t>(sel) & 3))) || !rnd ||
+        (reinterpret_cast<uintptr_t>(rnd) & 3) || !sel_out || (reinterpret_cast<uintptr_t>(sel_out) & 3))
+        return MOC_ERR_INVALID_ARG;
+    // F(i) accumulated in double from p_0 = exp(-lambda), p_i = p_{i-1} lambda / i
+    moc::PoissonThresholds thr{};
+    const double lam = double(lambda);
+    double p = std::exp(-lam), cdf = p;
+    for (int i = 0; i < m_max; ++i) {
+        if (i > 0) {
+            p = p * lam / double(i);
+            cdf = cdf + p;
+        }
+        const double v = std::floor(cdf * 4294967296.0);
+        thr.t[i] = v >= 4294967296.0 ? (uint64_t(1) << 32) : uint64_t(v);
+    }
+    return cuda_status(moc::launch_perturb(lay->dv, B * H, k, m_max, causal ? 1 : 0, sel, rnd, p_max, thr,
+                                           sel_out, (cudaStream_t)stream));
 }
 
 extern "C" size_t moc_attention_workspace_bytes(const moc_layout* lay, int B, int H, int d, int k) {

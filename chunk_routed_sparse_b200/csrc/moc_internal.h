@@ -83,4 +83,12 @@ cudaError_t launch_attend_tc(const DevLayout& dv, int BH, int d, const void* Q, 
 cudaError_t launch_merge(int BH, int L, int d, int k, const int32_t* sel, void* O, float* lse,
                          const char* ws, const WsPlan& p, cudaStream_t s);
 
+// Poisson distribution function at 0 .. m_max-1 scaled to 2^32 (drop-in counts)
+struct PoissonThresholds {
+    uint64_t t[kMaxK];
+};
+cudaError_t launch_perturb(const DevLayout& dv, int BH, int k, int m_max, int causal, const int32_t* sel,
+                           const uint32_t* rnd, float p_max, const PoissonThresholds& thr, int32_t* out,
+                           cudaStream_t s);
+
 }  // namespace moc

@@ -134,6 +134,28 @@ moc_status moc_pool_keys(const moc_layout* layout, int B, int H, int d, const vo
 moc_status moc_route(const moc_layout* layout, int B, int H, int d, const void* Q,
                      const float* Kbar, int k, int causal, int32_t* sel, moc_stream_t stream);
 
+/* (2') Training-time routing perturbations (Summary, appendix training
+ * details; [DL] slide 14): context drop-off and drop-in on a selection from
+ * (2). Per (b, h, query) - caption queries get all -1 - with the random draws
+ * given as data, rnd: device uint32 [B][H][L][2 + k + m_max]:
+ *   drop-off: n_drop = floor((rnd[0] / 2^32) * p_max * k) (fp64 products, left
+ *     to right; at most the number of selected chunks); the n_drop selected
+ *     entries with the smallest (rnd[2 + j], j) are removed;
+ *   drop-in: m = min(m_max, Poisson(lambda) inverted at rnd[1]) (the
+ *     distribution function is accumulated in fp64 from exp(-lambda) and
+ *     compared as floor(F * 2^32)); the a-th added chunk is entry
+ *     floor(rnd[2 + k + a] * n_left / 2^32) of the query's routing candidates
+ *     (same causal flag as (2)) that are neither in sel nor already added,
+ *     in ascending chunk order.
+ * sel: device int32 [B][H][L][k] from (2) (NULL when k == 0); sel_out: device
+ * int32 [B][H][L][k + m_max]: survivors in their original order, then the
+ * added chunks, -1 padded - a selection the attention calls take with
+ * k + m_max in place of k. 0 <= p_max <= 1, lambda >= 0 finite, m_max >= 0,
+ * 1 <= k + m_max <= 31. Deterministic. */
+moc_status moc_route_perturb(const moc_layout* layout, int B, int H, int k, int causal,
+                             const int32_t* sel, const uint32_t* rnd, float p_max, float lambda,
+                             int m_max, int32_t* sel_out, moc_stream_t stream);
+
 /* Bytes of device workspace moc_attention_fwd and the three stage calls need
  * for this problem (0 on invalid arguments). Holds the per-chunk query lists,
  * the scheduler's counters and the partial outputs (1+k fp32 rows of d plus
