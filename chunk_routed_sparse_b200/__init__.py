@@ -72,6 +72,8 @@ SIGNATURES = {
     "moc_forward_host": (_I, [_P, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _P, _P, _P, _SZ, _I, _P]),
     "moc_forward_host_device_bytes": (_SZ, [_P, _I, _I, _I, _I, _I]),
     "moc_route_perturb": (_I, [_P, _I, _I, _I, _I, _P, _P, _F, _F, _I, _P, _P]),
+    "moc_outer_route": (_I, [_P, _I, _I, _I, _P, _P, _I, _I, _P, _P]),
+    "moc_route_masked": (_I, [_P, _I, _I, _I, _P, _P, _I, _I, _P, _P, _P]),
 }
 
 
@@ -186,6 +188,30 @@ def route(layout: Layout, Q: torch.Tensor, kbar: torch.Tensor, k: int, causal: b
         out = torch.empty(B, H, L, k, dtype=torch.int32, device=Q.device)
     _check(lib().moc_route(layout.handle, B, H, d, _ptr(Q), _ptr(kbar), k, int(bool(causal)),
                            _ptr(out), _stream()), "moc_route")
+    return out
+
+
+def outer_route(layout: Layout, Qbar: torch.Tensor, Kbar: torch.Tensor, M: int, causal: bool = True,
+                out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Outer-loop routing (moc_outer_route): Qbar = pool_keys(layout, Q), Kbar =
+    pool_keys(layout, K), both fp32 [B, H, C, d]; returns int64 [B, H, G] masks
+    (bit s = segment s allowed)."""
+    B, H, C, d = Qbar.shape
+    G = len(layout.table(1)) // 2
+    if out is None:
+        out = torch.empty(B, H, G, dtype=torch.int64, device=Qbar.device)
+    _check(lib().moc_outer_route(layout.handle, B, H, d, _ptr(Qbar), _ptr(Kbar), M, 1 if causal else 0,
+                                 _ptr(out), _stream()), "moc_outer_route")
+    return out
+
+
+def route_masked(layout: Layout, Q: torch.Tensor, kbar: torch.Tensor, k: int, seg_mask: torch.Tensor,
+                 causal: bool = True, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    B, H, L, d = _dims(Q)
+    if out is None:
+        out = torch.empty(B, H, L, k, dtype=torch.int32, device=Q.device)
+    _check(lib().moc_route_masked(layout.handle, B, H, d, _ptr(Q), _ptr(kbar), k, 1 if causal else 0,
+                                  _ptr(seg_mask), _ptr(out), _stream()), "moc_route_masked")
     return out
 
 

@@ -89,7 +89,36 @@ extern "C" moc_status moc_route(const moc_layout* lay, int B, int H, int d, cons
         (reinterpret_cast<uintptr_t>(sel) & 3))
         return MOC_ERR_INVALID_ARG;
     return cuda_status(moc::launch_route(lay->dv, B * H, lay->total_rtiles, d, Q, Kbar, k,
-                                         causal ? 1 : 0, sel, (cudaStream_t)stream));
+                                         causal ? 1 : 0, nullptr, sel, (cudaStream_t)stream));
+}
+
+extern "C" moc_status moc_outer_route(const moc_layout* lay, int B, int H, int d, const float* Qbar,
+                                      const float* Kbar, int M, int causal, uint64_t* seg_mask,
+                                      moc_stream_t stream) {
+    moc_status st = check_common(lay, B, H, d, 0);
+    if (st != MOC_OK) return st;
+    if (M < 0) return MOC_ERR_INVALID_ARG;
+    if (lay->n_shots > 64) return MOC_ERR_UNSUPPORTED;  // one 64-bit mask per block
+    if (B * H == 0) return MOC_OK;
+    if (!Qbar || !Kbar || !seg_mask || (reinterpret_cast<uintptr_t>(Qbar) & 15) ||
+        (reinterpret_cast<uintptr_t>(Kbar) & 15) || (reinterpret_cast<uintptr_t>(seg_mask) & 7))
+        return MOC_ERR_INVALID_ARG;
+    return cuda_status(moc::launch_outer(lay->dv, B * H, d, Qbar, Kbar, M, causal ? 1 : 0, seg_mask,
+                                         (cudaStream_t)stream));
+}
+
+extern "C" moc_status moc_route_masked(const moc_layout* lay, int B, int H, int d, const void* Q,
+                                       const float* Kbar, int k, int causal, const uint64_t* seg_mask,
+                                       int32_t* sel, moc_stream_t stream) {
+    moc_status st = check_common(lay, B, H, d, k);
+    if (st != MOC_OK) return st;
+    if (lay->n_shots > 64) return MOC_ERR_UNSUPPORTED;
+    if (B * H == 0 || k == 0) return MOC_OK;
+    if (!Q || !Kbar || !sel || !seg_mask || !aligned16(Q) || !aligned16(Kbar) ||
+        (reinterpret_cast<uintptr_t>(sel) & 3) || (reinterpret_cast<uintptr_t>(seg_mask) & 7))
+        return MOC_ERR_INVALID_ARG;
+    return cuda_status(moc::launch_route(lay->dv, B * H, lay->total_rtiles, d, Q, Kbar, k,
+                                         causal ? 1 : 0, seg_mask, sel, (cudaStream_t)stream));
 }
 
 extern "C" moc_status moc_route_perturb(const moc_layout* lay, int B, int H, int k, int causal,

@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(256) perturb_kernel(DevLayout dv, int64_t rows
     // candidate is found by walking them once
     int m = 0;
     for (int i = 0; i < m_max; ++i) m += (thr.t[i] <= uint64_t(w[1])) ? 1 : 0;
-    int ex[kMaxK];
+    int ex[kMaxK] = {};
     int nex = 0;
     auto exclude = [&](int pos) {  // insert into the sorted list
         int i = nex++;

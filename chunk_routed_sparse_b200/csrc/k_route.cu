@@ -186,7 +186,7 @@ template <int D, int KMAX>
 __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
     route_tc_kernel(const __grid_constant__ CUtensorMap tmQ, DevLayout dv, int64_t total_tiles,
                     int64_t rtiles, const float* __restrict__ Kbar, int k, int causal,
-                    int32_t* __restrict__ sel) {
+                    const uint64_t* __restrict__ seg_mask, int32_t* __restrict__ sel) {
     using C = RCfg<D>;
     using WP = RWarps<KMAX>;
     constexpr int NWG = WP::kNwg, SLICE = WP::kSlice;
@@ -341,6 +341,7 @@ __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
                     for (int j = 0; j < k; ++j) out[size_t(row) * k + j] = -1;
                 continue;
             }
+            const uint64_t smask = seg_mask ? seg_mask[size_t(x.bh) * dv.G + x.g] : ~0ull;
             float ts[KMAX];
             int tj[KMAX];
 #pragma unroll
@@ -361,9 +362,17 @@ __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
                     tmem_ld32(lane_addr + c0, sc);
                     tmem_wait_ld_regs(sc);
                     const int pos0 = b * SLICE + c0;
+                    // columns of this chunk that take part (warp-uniform): those inside
+                    // the slice and, with an outer-loop mask, in a selected segment
+                    uint32_t allow = (nbc - c0 >= 32) ? 0xffffffffu : ((1u << (nbc - c0)) - 1u);
+                    if (seg_mask) {
+                        const bool ok = ((allow >> lane) & 1u) &&
+                                        ((smask >> dv.cand_seg[x.cbeg + pos0 + lane]) & 1ull);
+                        allow = __ballot_sync(0xffffffffu, ok);
+                    }
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
-                        if (c0 + e < nbc) topk_push<KMAX>(ts, tj, __uint_as_float(sc[e]), pos0 + e);
+                        if ((allow >> e) & 1u) topk_push<KMAX>(ts, tj, __uint_as_float(sc[e]), pos0 + e);
                 }
                 tc_fence_before();
                 mbar_arrive(bar(R_S_FREE + w));
@@ -388,7 +397,7 @@ __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
 
 template <int D, int KMAX>
 cudaError_t launch_dk(const DevLayout& dv, int BH, int64_t rtiles, const void* Q, const float* Kbar, int k,
-                      int causal, int32_t* sel, cudaStream_t s) {
+                      int causal, const uint64_t* seg_mask, int32_t* sel, cudaStream_t s) {
     CUtensorMap tmQ;
     if (!make_tmap(&tmQ, Q, D, int64_t(BH) * dv.L)) return cudaErrorInvalidValue;
     const int smem = RCfg<D>::kSmem;
@@ -399,33 +408,35 @@ cudaError_t launch_dk(const DevLayout& dv, int BH, int64_t rtiles, const void* Q
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t total = int64_t(BH) * rtiles;
     const int grid = int(total < sms ? total : sms);
-    route_tc_kernel<D, KMAX><<<grid, RWarps<KMAX>::kThreads, smem, s>>>(tmQ, dv, total, rtiles, Kbar, k, causal, sel);
+    route_tc_kernel<D, KMAX><<<grid, RWarps<KMAX>::kThreads, smem, s>>>(tmQ, dv, total, rtiles, Kbar, k, causal,
+                                                                        seg_mask, sel);
     return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t launch_d(const DevLayout& dv, int BH, int64_t rtiles, const void* Q, const float* Kbar, int k,
-                     int causal, int32_t* sel, cudaStream_t s) {
+                     int causal, const uint64_t* seg_mask, int32_t* sel, cudaStream_t s) {
     // exact list length for small k (the insertion network costs one level per entry)
     switch (k) {
-        case 1: return launch_dk<D, 1>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
-        case 2: return launch_dk<D, 2>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
-        case 3: return launch_dk<D, 3>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
-        case 4: return launch_dk<D, 4>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
+        case 1: return launch_dk<D, 1>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
+        case 2: return launch_dk<D, 2>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
+        case 3: return launch_dk<D, 3>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
+        case 4: return launch_dk<D, 4>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
         default: break;
     }
-    if (k <= 8) return launch_dk<D, 8>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
-    if (k <= 16) return launch_dk<D, 16>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
-    return launch_dk<D, 32>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
+    if (k <= 8) return launch_dk<D, 8>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
+    if (k <= 16) return launch_dk<D, 16>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
+    return launch_dk<D, 32>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
 }
 
 }  // namespace
 
 cudaError_t launch_route(const DevLayout& dv, int BH, int64_t rtiles, int d, const void* Q,
-                         const float* Kbar, int k, int causal, int32_t* sel, cudaStream_t s) {
+                         const float* Kbar, int k, int causal, const uint64_t* seg_mask, int32_t* sel,
+                         cudaStream_t s) {
     if (rtiles <= 0 || BH > 65535) return cudaErrorInvalidValue;
-    if (d == 128) return launch_d<128>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
-    return launch_d<64>(dv, BH, rtiles, Q, Kbar, k, causal, sel, s);
+    if (d == 128) return launch_d<128>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
+    return launch_d<64>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
 }
 
 }  // namespace moc

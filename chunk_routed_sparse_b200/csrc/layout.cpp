@@ -59,6 +59,8 @@ moc_status build_host(const moc_layout_desc* d, moc_layout* lay) {
     // each shot's video chunks must be one run of vid, frames non-decreasing
     std::vector<int32_t> run_lo(NV), run_hi(NV);
     std::set<int32_t> seen;
+    std::vector<int32_t> vseg(n, -1);  // segment (shot run, stream order) of every video chunk
+    lay->seg_voff.assign(1, 0);
     for (int v = 0; v < NV;) {
         int32_t s = lay->shot[vid[v]];
         if (seen.count(s)) return MOC_ERR_LAYOUT;  // shot split by another shot
@@ -68,10 +70,16 @@ moc_status build_host(const moc_layout_desc* d, moc_layout* lay) {
             if (w > v && lay->frame[vid[w]] < lay->frame[vid[w - 1]]) return MOC_ERR_LAYOUT;
             ++w;
         }
-        for (int x = v; x < w; ++x) { run_lo[x] = v; run_hi[x] = w; }
+        for (int x = v; x < w; ++x) {
+            run_lo[x] = v;
+            run_hi[x] = w;
+            vseg[vid[x]] = int32_t(lay->seg_voff.size()) - 1;
+        }
+        lay->seg_voff.push_back(w);
         v = w;
     }
     lay->n_shots = int32_t(seen.size());
+    lay->vid = vid;
 
     // anchor video range [alo, ahi) in vid-space of every video chunk
     std::vector<int32_t> alo(n, -1), ahi(n, -1);
@@ -114,9 +122,11 @@ moc_status build_host(const moc_layout_desc* d, moc_layout* lay) {
     lay->ar_off.assign(1, 0);
     lay->cand_off.assign(1, 0);
     lay->cand_ncausal.resize(G);
+    lay->grp_seg.assign(G, -1);
     lay->rtile_off.assign(1, 0);
     lay->ar.clear();
     lay->cand.clear();
+    lay->cand_seg.clear();
     lay->max_cand = 0;
     for (int g = 0; g < G; ++g) {
         const int c0 = groups[g].first, c1 = groups[g].second;
@@ -135,6 +145,9 @@ moc_status build_host(const moc_layout_desc* d, moc_layout* lay) {
             for (int v = 0; v < a; ++v) lay->cand.push_back(vid[v]);
             lay->cand_ncausal[g] = a;
             for (int v = b; v < NV; ++v) lay->cand.push_back(vid[v]);
+            for (int v = 0; v < a; ++v) lay->cand_seg.push_back(vseg[vid[v]]);
+            for (int v = b; v < NV; ++v) lay->cand_seg.push_back(vseg[vid[v]]);
+            lay->grp_seg[g] = vseg[c0];
         }
         std::sort(rng.begin(), rng.end());
         std::vector<std::pair<int32_t, int32_t>> merged;
@@ -177,7 +190,7 @@ moc_status upload(moc_layout* lay) {
     std::vector<const std::vector<int32_t>*> tabs = {
         &lay->chunk_off, &lay->grp_q0, &lay->grp_q1, &lay->grp_kind, &lay->ar_off, &lay->ar,
         &lay->cand_off, &lay->cand, &lay->cand_ncausal, &lay->rtile_off, &lay->atile_off,
-        &lay->a_order};
+        &lay->a_order, &lay->cand_seg, &lay->grp_seg, &lay->seg_voff, &lay->vid};
     std::vector<size_t> offs;
     size_t total = 0;
     for (auto* t : tabs) {
@@ -216,6 +229,11 @@ moc_status upload(moc_layout* lay) {
     dv.rtile_off = at(9);
     dv.atile_off = at(10);
     dv.a_order = at(11);
+    dv.S = lay->n_shots;
+    dv.cand_seg = at(12);
+    dv.grp_seg = at(13);
+    dv.seg_voff = at(14);
+    dv.vid = at(15);
     dv.err = reinterpret_cast<int32_t*>(static_cast<char*>(lay->dev_block) + err_off);
     return MOC_OK;
 }

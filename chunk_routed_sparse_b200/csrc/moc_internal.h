@@ -31,6 +31,11 @@ struct DevLayout {
     const int32_t* rtile_off;    // [G+1] prefix of router tiles (kQTile queries) per group
     const int32_t* atile_off;    // [G+1] prefix of anchor items (kItemRows queries), groups in a_order
     const int32_t* a_order;      // [G] groups by descending anchor keys per tile
+    int32_t S;                   // segments (shots) in stream order
+    const int32_t* cand_seg;     // segment of every entry of cand
+    const int32_t* grp_seg;      // [G] segment of the group's queries (-1: caption group)
+    const int32_t* seg_voff;     // [S+1] offsets into vid of every segment's video chunks
+    const int32_t* vid;          // video chunk ids in stream order
     int32_t* err;                // [2] error word + detail of kernels without a workspace (router)
 };
 
@@ -46,6 +51,7 @@ struct moc_layout {
     std::vector<int32_t> chunk_off, kind, shot, frame;
     std::vector<int32_t> grp_q0, grp_q1, grp_kind, ar_off, ar, cand_off, cand, cand_ncausal;
     std::vector<int32_t> rtile_off, atile_off, a_order;
+    std::vector<int32_t> cand_seg, grp_seg, seg_voff, vid;  // segments (shots) in stream order
     std::vector<int64_t> grp_keys;  // anchor keys of each group
     void* dev_block = nullptr;
     moc::DevLayout dv{};
@@ -74,7 +80,10 @@ enum { ERR_NONE = 0, ERR_TIMEOUT = 1, ERR_CHECK = 2 };
 cudaError_t launch_pool(const DevLayout& dv, int BH, int d, const void* K, float* Kbar,
                         cudaStream_t s);
 cudaError_t launch_route(const DevLayout& dv, int BH, int64_t rtiles, int d, const void* Q,
-                         const float* Kbar, int k, int causal, int32_t* sel, cudaStream_t s);
+                         const float* Kbar, int k, int causal, const uint64_t* seg_mask, int32_t* sel,
+                         cudaStream_t s);
+cudaError_t launch_outer(const DevLayout& dv, int BH, int d, const float* Qbar, const float* Kbar, int M,
+                         int causal, uint64_t* seg_mask, cudaStream_t s);
 cudaError_t launch_qlists(const DevLayout& dv, int BH, int k, const int32_t* sel, char* ws,
                           const WsPlan& p, cudaStream_t s);
 cudaError_t launch_attend_tc(const DevLayout& dv, int BH, int d, const void* Q, const void* K,

@@ -134,6 +134,29 @@ moc_status moc_pool_keys(const moc_layout* layout, int B, int H, int d, const vo
 moc_status moc_route(const moc_layout* layout, int B, int H, int d, const void* Q,
                      const float* Kbar, int k, int causal, int32_t* sel, moc_stream_t stream);
 
+/* (2'') Outer-loop context routing (Summary, appendix I): a coarse router
+ * picks, per query block, the top-M context segments the inner router may
+ * select from. Segments are the shots' video chunks, numbered 0..S-1 in stream
+ * order (S <= 64); a query block is a query group of the layout (queries
+ * sharing one anchor set; table 1 of moc_layout_table lists them, G of them).
+ * Features are token means - the block's queries and the segment's keys -
+ * formed from per-chunk means (Qbar from moc_pool_keys applied to Q, Kbar from
+ * (1)) weighted by chunk length, in fp32; score = unscaled dot product.
+ * Candidates are the other segments (with causal != 0 only earlier ones); top-M
+ * by (score descending, segment ascending), all when fewer than M. seg_mask:
+ * device uint64 [B][H][G], bit s set = segment s allowed; the block's own
+ * segment is always set (mandatory context); caption blocks get 0. */
+moc_status moc_outer_route(const moc_layout* layout, int B, int H, int d, const float* Qbar,
+                           const float* Kbar, int M, int causal, uint64_t* seg_mask,
+                           moc_stream_t stream);
+
+/* (2) restricted by an outer-loop mask: as moc_route, with a query's
+ * candidates limited to chunks of segments whose bit is set in its block's
+ * seg_mask (from moc_outer_route). */
+moc_status moc_route_masked(const moc_layout* layout, int B, int H, int d, const void* Q,
+                            const float* Kbar, int k, int causal, const uint64_t* seg_mask,
+                            int32_t* sel, moc_stream_t stream);
+
 /* (2') Training-time routing perturbations (Summary, appendix training
  * details; [DL] slide 14): context drop-off and drop-in on a selection from
  * (2). Per (b, h, query) - caption queries get all -1 - with the random draws
