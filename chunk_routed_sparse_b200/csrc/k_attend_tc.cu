@@ -420,17 +420,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int c = 0; c < kKT; ++c)
                         if (c >= nvalid) s[c] = __float_as_uint(-INFINITY);
                 }
-                // row max of the raw scores (the positive scale commutes with max)
-                float a0 = __uint_as_float(s[0]), a1 = __uint_as_float(s[1]);
-                float a2 = __uint_as_float(s[2]), a3 = __uint_as_float(s[3]);
+                // row max of the raw scores (the positive scale commutes with max), as
+                // eight independent 3-input max chains
+                float a[8];
 #pragma unroll
-                for (int c = 4; c < kKT; c += 8) {
-                    a0 = max3(a0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
-                    a1 = max3(a1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
-                    a2 = max3(a2, __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));
-                    a3 = max3(a3, __uint_as_float(s[c + 6]), __uint_as_float(s[c + 7]));
+                for (int i = 0; i < 8; ++i) a[i] = fmaxf(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1]));
+#pragma unroll
+                for (int c = 16; c < kKT; c += 16) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) a[i] = max3(a[i], __uint_as_float(s[c + 2 * i]), __uint_as_float(s[c + 2 * i + 1]));
                 }
-                const float mx = max3(a0, a1, fmaxf(a2, a3)) * scale_log2;  // log2 units
+                const float mx = max3(max3(a[0], a[1], a[2]), max3(a[3], a[4], a[5]), fmaxf(a[6], a[7])) * scale_log2;
                 float alpha = 1.f;
                 bool rescale = false;
                 if (j == 0) {
