@@ -73,7 +73,23 @@ enum { R_Q_FULL = 0, R_Q_EMPTY = 4, R_S_FULL = 8, R_S_FREE = 12, R_KB_FREE = 16,
 struct RShared {  // at oBar + 192 (after the barriers)
     uint32_t tmem_base;
     int abort;
+    int64_t t_beg, t_end;  // this CTA's tile range
 };
+
+// First global tile t (head-major) whose cost prefix reaches `target`; tile costs
+// are positive, so the prefix strictly increases.
+__device__ int64_t tile_at_cost(const DevLayout& dv, int64_t rtiles, int causal, int64_t total_tiles,
+                                int64_t target) {
+    const int32_t* pre = dv.rcost[causal ? 1 : 0];
+    const int64_t head = pre[rtiles];
+    int64_t lo = 0, hi = total_tiles;
+    while (lo < hi) {
+        const int64_t mid = (lo + hi) >> 1;
+        const int64_t cum = (mid / rtiles) * head + pre[mid % rtiles];
+        if (cum >= target) hi = mid; else lo = mid + 1;
+    }
+    return lo;
+}
 
 // Insert (cs, cj) into a register list sorted by descending score (branch
 // free: per entry one compare, a max / min pair for the scores and two
@@ -202,9 +218,6 @@ __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
     auto bar = [&](int i) { return sBar + 8u * uint32_t(i); };
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    // this CTA's contiguous range of tiles
-    const int64_t t_beg = total_tiles * blockIdx.x / gridDim.x;
-    const int64_t t_end = total_tiles * (blockIdx.x + 1) / gridDim.x;
 
     if (tid == 0) {
         for (int x = 0; x < C::kQStages; ++x) {
@@ -218,6 +231,10 @@ __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
         mbar_init(bar(R_KB_FREE), 1);
         mbar_init(bar(R_MMA_DONE), 1);
         sh.abort = 0;
+        // this CTA's contiguous range of tiles: equal shares of the estimated work
+        const int64_t total_cost = (total_tiles / rtiles) * int64_t(dv.rcost[causal ? 1 : 0][rtiles]);
+        sh.t_beg = tile_at_cost(dv, rtiles, causal, total_tiles, total_cost * blockIdx.x / gridDim.x);
+        sh.t_end = tile_at_cost(dv, rtiles, causal, total_tiles, total_cost * (blockIdx.x + 1) / gridDim.x);
         fence_mbar_init();
     }
     if (warp == WP::kIssuer) {
@@ -228,6 +245,7 @@ __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sh.tmem_base;
+    const int64_t t_beg = sh.t_beg, t_end = sh.t_end;
 
     if (warp == WP::kProducer) {
         // ------------------------------------------------------------ Q producer

@@ -171,6 +171,24 @@ moc_status build_host(const moc_layout_desc* d, moc_layout* lay) {
         lay->rtile_off.push_back(lay->rtile_off.back() + (nq + moc::kQTile - 1) / moc::kQTile);
     }
     lay->total_rtiles = lay->rtile_off.back();
+    // estimated cost of every router tile, for splitting the tiles into contiguous
+    // per-CTA ranges of equal work: a fixed part for a tile that has candidates (Q
+    // stream, MMAs) plus a quarter per candidate (the per-row top-k); 1 for a tile
+    // without candidates (its rows are only written)
+    lay->rcost_full.assign(1, 0);
+    lay->rcost_causal.assign(1, 0);
+    for (int g = 0; g < G; ++g) {
+        const int32_t ntile = lay->rtile_off[g + 1] - lay->rtile_off[g];
+        const bool video = lay->grp_kind[g] == MOC_VIDEO;
+        const int32_t nfull = video ? lay->cand_off[g + 1] - lay->cand_off[g] : 0;
+        const int32_t ncaus = video ? lay->cand_ncausal[g] : 0;
+        const int32_t cf = nfull > 0 ? 8 + (nfull + 3) / 4 : 1;
+        const int32_t cc = ncaus > 0 ? 8 + (ncaus + 3) / 4 : 1;
+        for (int32_t i = 0; i < ntile; ++i) {
+            lay->rcost_full.push_back(lay->rcost_full.back() + cf);
+            lay->rcost_causal.push_back(lay->rcost_causal.back() + cc);
+        }
+    }
     // anchor work items of kItemRows queries: groups with the most keys first (longest work first)
     lay->a_order.resize(G);
     std::iota(lay->a_order.begin(), lay->a_order.end(), 0);
@@ -190,7 +208,8 @@ moc_status upload(moc_layout* lay) {
     std::vector<const std::vector<int32_t>*> tabs = {
         &lay->chunk_off, &lay->grp_q0, &lay->grp_q1, &lay->grp_kind, &lay->ar_off, &lay->ar,
         &lay->cand_off, &lay->cand, &lay->cand_ncausal, &lay->rtile_off, &lay->atile_off,
-        &lay->a_order, &lay->cand_seg, &lay->grp_seg, &lay->seg_voff, &lay->vid};
+        &lay->a_order, &lay->cand_seg, &lay->grp_seg, &lay->seg_voff, &lay->vid,
+        &lay->rcost_full, &lay->rcost_causal};
     std::vector<size_t> offs;
     size_t total = 0;
     for (auto* t : tabs) {
@@ -234,6 +253,8 @@ moc_status upload(moc_layout* lay) {
     dv.grp_seg = at(13);
     dv.seg_voff = at(14);
     dv.vid = at(15);
+    dv.rcost[0] = at(16);
+    dv.rcost[1] = at(17);
     dv.err = reinterpret_cast<int32_t*>(static_cast<char*>(lay->dev_block) + err_off);
     return MOC_OK;
 }

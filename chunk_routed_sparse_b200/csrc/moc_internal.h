@@ -36,6 +36,7 @@ struct DevLayout {
     const int32_t* grp_seg;      // [G] segment of the group's queries (-1: caption group)
     const int32_t* seg_voff;     // [S+1] offsets into vid of every segment's video chunks
     const int32_t* vid;          // video chunk ids in stream order
+    const int32_t* rcost[2];     // [rtiles+1] prefix of estimated router tile costs, full / causal lists
     int32_t* err;                // [2] error word + detail of kernels without a workspace (router)
 };
 
@@ -52,6 +53,7 @@ struct moc_layout {
     std::vector<int32_t> grp_q0, grp_q1, grp_kind, ar_off, ar, cand_off, cand, cand_ncausal;
     std::vector<int32_t> rtile_off, atile_off, a_order;
     std::vector<int32_t> cand_seg, grp_seg, seg_voff, vid;  // segments (shots) in stream order
+    std::vector<int32_t> rcost_full, rcost_causal;          // router tile cost prefixes
     std::vector<int64_t> grp_keys;  // anchor keys of each group
     void* dev_block = nullptr;
     moc::DevLayout dv{};
