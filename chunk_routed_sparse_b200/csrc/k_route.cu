@@ -10,7 +10,9 @@
 //
 // Work unit: a 128-query tile of one query group (all its queries share one
 // candidate list) times a block of the group's candidates. One persistent CTA
-// per SM walks a contiguous range of tiles with NWG selection warpgroups
+// per SM walks a contiguous range of tiles - the ranges split the tiles by the
+// layout's estimated per-tile cost, so CTAs holding the tiles of late shots
+// (many candidates) take fewer of them - with NWG selection warpgroups
 // (4 for k <= 8, else 2) and two more warps:
 //   warp 4*NWG (one lane): streams each tile's Q rows (two 64-column,
 //          128-byte-swizzled slabs) into a 2-stage ring with TMA;
