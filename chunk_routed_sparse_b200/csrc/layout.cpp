@@ -339,6 +339,12 @@ extern "C" moc_status moc_layout_table(const moc_layout* layout, int which, int3
         case 4: src = &layout->cand; break;
         case 5: src = &layout->cand_off; break;
         case 6: src = &layout->cand_ncausal; break;
+        case 7: src = &layout->cand_seg; break;
+        case 8: src = &layout->grp_seg; break;
+        case 9: src = &layout->seg_voff; break;
+        case 10: src = &layout->vid; break;
+        case 11: src = &layout->rcost_full; break;
+        case 12: src = &layout->rcost_causal; break;
         default: return MOC_ERR_INVALID_ARG;
     }
     *count = int64_t(src->size());

@@ -107,7 +107,12 @@ moc_status moc_layout_info(const moc_layout* layout, int64_t* L, int32_t* C, int
  *        2 group anchor key ranges as (start,end) pairs in group order,
  *        3 anchor range offsets per group [G+1], 4 candidate chunk ids in
  *        group order, 5 candidate offsets per group [G+1],
- *        6 causal candidate count per group [G].
+ *        6 causal candidate count per group [G], 7 segment (shot, numbered in
+ *        stream order) of every candidate in table 4, 8 segment of every
+ *        group's queries [G] (-1: caption group), 9 offsets of every segment's
+ *        video chunks in table 10 [S+1], 10 video chunk ids in stream order,
+ *        11 / 12 prefix of the router's estimated tile costs for the full /
+ *        causal candidate lists [router tiles + 1].
  * Writes min(count, cap) int32 values to out (may be NULL with cap 0) and
  * the full count to *count. */
 moc_status moc_layout_table(const moc_layout* layout, int which, int32_t* out, int64_t cap,

@@ -151,3 +151,31 @@ def test_layout_info_counts_shots():
     assert lay.n_shots == 8
     lay1 = _host_layout(W.single())
     assert lay1.n_shots == 1
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged", "eight"])
+def test_segment_tables_agree_with_oracle(name):
+    """Segments (shots in stream order) as the outer router and the masked
+    router see them, against the oracle's own segmentation and roles."""
+    from oracle import outer as OU
+    wl = W.CONFIGS[name]()
+    lay = _host_layout(wl)
+    orc = oracle.Layout(wl)
+    seg = OU.segments(orc)
+    cand, cand_off = lay.table(4), lay.table(5)
+    cand_seg, grp_seg = lay.table(7), lay.table(8)
+    seg_voff, vid = lay.table(9), lay.table(10)
+    assert len(seg_voff) == int(seg.max()) + 2 and vid == [c for c in range(orc.C) if orc.kind[c] == 1]
+    for s_ in range(len(seg_voff) - 1):
+        assert all(seg[c] == s_ for c in vid[seg_voff[s_]:seg_voff[s_ + 1]])
+    assert cand_seg == [int(seg[c]) for c in cand]
+    grp = lay.table(1)
+    for g in range(len(grp) // 2):
+        c0 = int(orc.chunk_of_token[grp[2 * g]])
+        assert grp_seg[g] == (int(seg[c0]) if orc.kind[c0] == 1 else -1)
+    # router tile cost prefixes: increasing, one entry per router tile plus one
+    for which in (11, 12):
+        pre = lay.table(which)
+        assert pre[0] == 0 and all(b > a for a, b in zip(pre, pre[1:]))
+        ntiles = sum((grp[2 * g + 1] - grp[2 * g] + 127) // 128 for g in range(len(grp) // 2))
+        assert len(pre) == ntiles + 1
