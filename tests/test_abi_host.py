@@ -45,7 +45,27 @@ WORKLOADS = [W.tiny(), W.single(), W.eight(), W.ragged(), W.stress(),
              W.ragged().replace(anchor="local", radius=2)]
 
 
-@pytest.mark.parametrize("wl", WORKLOADS, ids=lambda w: f"{w.name}-{w.anchor}")
+def _random_workload(rng, i):
+    """A random valid scene: 1-6 shots of 1-5 frames, each frame cut into 1-3
+    sub-chunks of 1-50 tokens, caption segments of 1-30 tokens placed before
+    shots at random (sometimes several in a row, sometimes none), any anchor
+    mode, radius 0-2, causal on or off."""
+    segs = []
+    for s in range(rng.integers(1, 7)):
+        for _ in range(rng.integers(0, 3)):
+            segs.append(W.Segment(int(rng.integers(1, 31)), W.CAPTION, s, -1))
+        for f in range(rng.integers(1, 6)):
+            for _ in range(rng.integers(1, 4)):
+                segs.append(W.Segment(int(rng.integers(1, 51)), W.VIDEO, s, f))
+    anchor = ["shot", "local", "chunk"][int(rng.integers(0, 3))]
+    return W.custom(f"rand{i}", 1, 1, 64, segs, anchor, int(rng.integers(0, 3)), bool(rng.integers(0, 2)),
+                    2, 7, "none")
+
+
+RANDOM = [_random_workload(np.random.default_rng(1000 + i), i) for i in range(120)]
+
+
+@pytest.mark.parametrize("wl", WORKLOADS + RANDOM, ids=lambda w: f"{w.name}-{w.anchor}")
 def test_layout_tables_agree_with_oracle_roles(wl):
     lay = _host_layout(wl)
     orc = oracle.Layout(wl)
@@ -153,12 +173,12 @@ def test_layout_info_counts_shots():
     assert lay1.n_shots == 1
 
 
-@pytest.mark.parametrize("name", ["tiny", "ragged", "eight"])
-def test_segment_tables_agree_with_oracle(name):
+@pytest.mark.parametrize("wl", [W.tiny(), W.ragged(), W.eight()] + RANDOM[:60],
+                         ids=lambda w: f"{w.name}-{w.anchor}")
+def test_segment_tables_agree_with_oracle(wl):
     """Segments (shots in stream order) as the outer router and the masked
     router see them, against the oracle's own segmentation and roles."""
     from oracle import outer as OU
-    wl = W.CONFIGS[name]()
     lay = _host_layout(wl)
     orc = oracle.Layout(wl)
     seg = OU.segments(orc)
