@@ -22,8 +22,10 @@
  *    library allocates device memory only inside moc_build_layout (its tables,
  *    freed by moc_layout_destroy); no hot-path call allocates.
  *  - Compute calls are asynchronous on the given stream and return after
- *    enqueueing. Argument errors are returned before anything is enqueued;
- *    a launch failure returns MOC_ERR_CUDA. No call throws across the ABI.
+ *    enqueueing (except moc_forward_host, which takes host buffers and returns
+ *    once its host outputs are complete). Argument errors are returned before
+ *    anything is enqueued; a launch failure returns MOC_ERR_CUDA. No call
+ *    throws across the ABI.
  *  - Limits: 1 <= C <= 16384 chunks, L < 2^26, B*H <= 65535, B*H*L*max(k,1) < 2^31,
  *    0 <= k <= 31, every chunk non-empty.
  */
