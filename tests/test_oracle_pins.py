@@ -265,3 +265,22 @@ def test_near_tie_rule():
     assert oracle.is_near(s[0], s[1], a[0], a[1])
     assert not oracle.is_near(s[0], s[2], a[0], a[2])
     assert oracle.is_near(s[2], s[3], a[2], a[3])     # guarded by magnitude
+
+
+def test_dense_comparison_layouts():
+    """The benchmark's dense and FLOP-matched block-diagonal layouts (k = 0):
+    the oracle's kept-pair counts are L^2 and the block sum of squares, and the
+    block-diagonal one matches the eight-shot scene's MoC count within 0.02 %."""
+    wl = W.eight()
+    L = wl.L
+    n_cap = sum(s.length for s in wl.segments if s.kind == W.CAPTION)
+    dense = [W.Segment(n_cap, W.CAPTION, -1, -1)] + \
+        [W.Segment(1500, W.VIDEO, 0, f) for f in range((L - n_cap) // 1500)]
+    blocks = [W.Segment(28405, W.VIDEO, s, 0) for s in range(6)] + [W.Segment(L - 6 * 28405, W.VIDEO, 6, 0)]
+    for segs, want in ((dense, L * L), (blocks, sum(s.length ** 2 for s in blocks))):
+        w2 = W.custom("cmp", 1, 1, 128, segs, "shot", 0, True, 0, 1, "none")
+        assert w2.L == L
+        lay = oracle.Layout(w2)
+        assert oracle.kept_pairs(w2, np.full((L, 0), -1, dtype=np.int32), lay) == want
+    moc_pairs = 4_943_332_144
+    assert abs(sum(s.length ** 2 for s in blocks) - moc_pairs) < 2e-4 * moc_pairs
