@@ -37,7 +37,7 @@ def _worker(rank, world, port, out):
 
 def test_ranks_get_independent_scenes_and_max_times():
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:  # no fork of this multi-threaded process
         out = m.dict()
         mp.start_processes(_worker, args=(2, port, out), nprocs=2, start_method="spawn")
         r0, r1 = out[0], out[1]
