@@ -7,10 +7,14 @@ than L2 (3 x 1.1 GB), so no L2 flush is needed between steps.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--config eight|single|tiny|ragged|stress] [--k K]
+                  [--shard heads|replicas] [--gather]
 
-Under torchrun every rank runs its own independent scene (weak scaling: the
-per-GPU work is fixed); there is no collective on the data path. Times are
-CUDA-event device times, max over ranks.
+Under torchrun (N > 1) the ranks split one scene's B*H (b, h) slices into
+contiguous shares (``--shard heads``, the default: strong scaling, the total
+work is fixed) or each run an independent scene (``--shard replicas``: weak
+scaling). Every stage is independent per slice, so neither has a collective on
+the data path; ``--gather`` all-gathers the output shares afterwards, outside
+the timed regions. Times are CUDA-event device times, max over ranks.
 """
 from __future__ import annotations
 
@@ -53,6 +57,12 @@ def workload(name: str, k, heads=None):
     if heads is not None:  # fewer heads of the same scene (profiling captures)
         wl = wl.replace(H=heads)
     return wl.with_k(k) if k is not None else wl
+
+
+def workload_string(wl, C: int) -> str:
+    """The workload name both arms print in config.workload."""
+    return (f"{wl.name}: B={wl.B} H={wl.H} L={wl.L} d={wl.d} k={wl.k} chunks={C} "
+            f"anchor={wl.anchor} causal={wl.causal}")
 
 
 def dist_env():
@@ -137,16 +147,16 @@ def kernel_traffic():
     return float(vals["dram_bytes_per_launch_full_scene"])
 
 
-def selected_pairs(layout_tables, wl, sel: torch.Tensor) -> int:
-    """Kept (query, key) pairs of the whole problem: anchor pairs from the
-    layout's group key counts plus the sizes of the selected chunks."""
+def selected_pairs(layout_tables, n_slices: int, wl, sel: torch.Tensor) -> int:
+    """Kept (query, key) pairs of ``n_slices`` (b, h) slices: anchor pairs from
+    the layout's group key counts plus the sizes of the selected chunks."""
     grp, ar, ar_off = layout_tables
     anchor = 0
     for g in range(len(grp) // 2):
         nq = grp[2 * g + 1] - grp[2 * g]
         keys = sum(ar[2 * x + 1] - ar[2 * x] for x in range(ar_off[g], ar_off[g + 1]))
         anchor += nq * keys
-    anchor *= wl.B * wl.H
+    anchor *= n_slices
     ln = torch.tensor([s.length for s in wl.segments], dtype=torch.int64, device=sel.device)
     routed = int(ln[sel[sel >= 0].long()].sum().item()) if sel.numel() else 0
     return anchor + routed
@@ -155,6 +165,42 @@ def selected_pairs(layout_tables, wl, sel: torch.Tensor) -> int:
 def scene_for_rank(wl, rank: int):
     """Weak scaling: every rank runs an independent scene of the same shape."""
     return wl.replace(seed=wl.seed + 1000 * rank)
+
+
+def sum_over_ranks(values, device=None):
+    """Element-wise sum of a list of floats over all ranks (identity at N=1)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return [float(v) for v in t.tolist()]
+
+
+def shard_slices(B: int, H: int, world: int, rank: int):
+    """Contiguous share [s0, s1) of the B*H flat (b, h) slices for one rank:
+    every slice belongs to exactly one rank and the shares differ by at most
+    one slice. Every stage of the path is independent per slice (the
+    jxzklqfsx.com MoC write-up, "計算效率": all operations are
+    head-independent), so the shares run with no exchange."""
+    n = B * H
+    base, extra = divmod(n, world)
+    s0 = rank * base + min(rank, extra)
+    return s0, s0 + base + (1 if rank < extra else 0)
+
+
+def gather_slices(part: torch.Tensor, n_slices: int, world: int) -> torch.Tensor:
+    """All-gather the per-rank slice shares ([s1 - s0, ...] each, in rank
+    order) into the whole [n_slices, ...] tensor on every rank. Shares are
+    padded to the largest one for the collective and trimmed after."""
+    import torch.distributed as dist
+    sizes = [shard_slices(1, n_slices, world, r) for r in range(world)]
+    mx = max(b - a for a, b in sizes)
+    buf = torch.zeros((mx,) + tuple(part.shape[1:]), dtype=part.dtype, device=part.device)
+    buf[:part.shape[0]].copy_(part)
+    out = torch.empty((world * mx,) + tuple(part.shape[1:]), dtype=part.dtype, device=part.device)
+    dist.all_gather_into_tensor(out, buf)
+    return torch.cat([out[r * mx:r * mx + (b - a)] for r, (a, b) in enumerate(sizes)])
 
 
 def max_over_ranks(values, device=None):
@@ -177,9 +223,21 @@ def run_ours(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    wl = scene_for_rank(workload(args.config, args.k, args.heads), rank)
-    B, H, L, d, k = wl.B, wl.H, wl.L, wl.d, wl.k
-    Qh, Kh, Vh = W.make_qkv(wl)
+    shard = args.shard if ws_ > 1 else "none"
+    if shard == "heads":
+        # one scene; this rank runs its share of the (b, h) slices (every stage is
+        # independent per slice and the layout is shared, so a share runs as B=1,
+        # H = its slice count)
+        wl = workload(args.config, args.k, args.heads)
+        s0, s1 = shard_slices(wl.B, wl.H, ws_, rank)
+        Qh, Kh, Vh = W.make_qkv_slices(wl, s0, s1)
+        B, H = 1, s1 - s0
+    else:
+        wl = scene_for_rank(workload(args.config, args.k, args.heads), rank)
+        s0, s1 = 0, wl.B * wl.H
+        Qh, Kh, Vh = W.make_qkv(wl)
+        B, H = wl.B, wl.H
+    L, d, k = wl.L, wl.d, wl.k
     Qh, Kh, Vh = Qh.pin_memory(), Kh.pin_memory(), Vh.pin_memory()
     dev = torch.device("cuda", local)
     Q, K, V = (t.to(dev, non_blocking=False) for t in (Qh, Kh, Vh))
@@ -210,7 +268,7 @@ def run_ours(args):
         step()
     moc.check_device_error(ws)
     torch.cuda.synchronize()
-    pairs = selected_pairs((lay.table(1), lay.table(2), lay.table(3)), wl, sel)
+    pairs = selected_pairs((lay.table(1), lay.table(2), lay.table(3)), B * H, wl, sel)
     flops = 4.0 * d * pairs
 
     def barrier():
@@ -244,7 +302,7 @@ def run_ours(args):
     moc.forward_host(lay, Qh, Kh, Vh, k, causal=wl.causal, scale=scale, dev=devbuf, out=Oh,
                      want_lse=False)  # untimed first call
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2e_steps = max(1, min(args.steps, 5))
+    e2e_steps = args.steps
     barrier()
     torch.cuda.synchronize()
     e0.record(stream)
@@ -257,40 +315,61 @@ def run_ours(args):
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
     del devbuf
 
+    gather = None
+    if shard == "heads" and args.gather:
+        # the whole O on every rank, outside the timed regions (NCCL all-gather of
+        # the slice shares, which sit in rank order in the [B*H, L, d] layout)
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        O_all = gather_slices(O.view(H, L, d), wl.B * wl.H, ws_)
+        g1.record(stream)
+        torch.cuda.synchronize()
+        gather = {"ms": g0.elapsed_time(g1), "bytes_per_rank_in": O.numel() * 2,
+                  "shape": list(O_all.shape)}
+        del O_all
+
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
+    job_pairs = int(sum_over_ranks([float(pairs)], dev)[0])
 
     ms_per_step = total_ms / args.steps
     tokens = B * L
+    # whole-job tokens per step: the head shares of one scene add up to that scene;
+    # replicas each run a scene of their own
+    job_tokens = wl.B * L if shard == "heads" else ws_ * tokens
     peaks, peak_src = load_peaks()
     att_s = stage_ms["attend"] / 1e3
     achieved_tf = flops / att_s / 1e12
     peak_tf = float(peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"]))
     traffic = kernel_traffic()
-    dense_pairs = B * H * L * L
+    # dense pairs of everything the job computed (the whole scene for a head split)
+    dense_pairs = (wl.B * wl.H if shard == "heads" else ws_ * B * H) * L * L
+    parallelism = {"none": "single GPU",
+                   "heads": f"head split x{ws_}: slices [{s0}, {s1}) of {wl.B * wl.H} on rank {rank}; "
+                            "no collective on the data path",
+                   "replicas": f"replicas x{ws_} (independent scenes, no collective)"}[shard]
     line = {
         "metric": METRIC,
-        "value": ws_ * tokens / (ms_per_step / 1e3),
+        "value": job_tokens / (ms_per_step / 1e3),
         "unit": "tokens/s",
         "n_gpus": ws_,
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": ms_per_step,
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if shard == "heads" else "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) + per-shot/per-frame mean offsets; no dataset)",
-        "config": {"workload": f"{wl.name}: B={B} H={H} L={L} d={d} k={k} chunks={lay.C} "
-                               f"anchor={wl.anchor} causal={wl.causal}",
-                   "tokens_per_step_per_gpu": tokens,
+        "config": {"workload": workload_string(wl, lay.C),
+                   "tokens_per_step_per_gpu": tokens if shard != "heads" else wl.B * L * H / (wl.B * wl.H),
                    "l2": "inputs larger than L2 (3 x %.2f GB), no flush" % (Q.numel() * 2 / 1e9),
-                   "parallelism": f"replicas x{ws_} (independent scenes, no collective)"},
+                   "parallelism": parallelism},
         "selected_pair_tflops_attend": achieved_tf,
-        "selected_pair_tflops_step": flops / (ms_per_step / 1e3) / 1e12,
+        "selected_pair_tflops_step": 4.0 * d * job_pairs / (ms_per_step / 1e3) / 1e12,
         "pct_bf16_peak_attend": 100.0 * achieved_tf / peak_tf,
         "stage_ms": stage_ms,
-        "pruned_fraction": 1.0 - pairs / dense_pairs,
-        "kept_pairs": pairs,
+        "pruned_fraction": 1.0 - job_pairs / dense_pairs,
+        "kept_pairs": job_pairs,
         "roofline": {"bound": "tensor", "kernel": "attend (4)", "achieved": achieved_tf,
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved_tf / peak_tf,
                      "peak_kind": f"bf16_tflops_sustained ({peak_src})",
@@ -299,17 +378,20 @@ def run_ours(args):
         "hbm_kernels": hbm_fracs(stage_ms, B, H, L, lay.C, d, k, peaks, routed_rows(lay, wl),
                                  int((sel >= 0).sum().item()) if k > 0 else 0),
         "clocks": clk,
-        "e2e": {"value": ws_ * tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+        "e2e": {"value": job_tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                 "ms_per_step": e2e_ms,
                 "path": "moc_forward_host: host buffers, 12 chunks of heads, copies overlapped",
                 "h2d_bytes_per_step": 3 * Q.numel() * 2, "d2h_bytes_per_step": O.numel() * 2},
         "gpu_launches": args.steps * sum(LAUNCHES_PER_STEP.values()),
     }
+    if gather is not None:
+        line["gather"] = gather
     if ws_ == 1 and not args.no_dense_compare and wl.name == "eight":
         line["dense_compare"] = dense_compare(moc, wl, Q, K, V, O, lse, stream, pairs,
                                               stage_ms, ms_per_step, peak_tf)
     if rank == 0 and ws_ == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, Qh, Kh, Vh, budget_s=args.cpu_budget)
+        line["routing_check"] = routing_check(wl, Qh, Kh, sel.cpu().numpy())
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws_ > 1:
@@ -432,9 +514,52 @@ def cpu_baseline(wl, Qh, Kh, Vh, budget_s: float = 20.0, rows_per_round: int = 6
                       f"heads x {lay.L} rows"}
 
 
+def routing_check(wl, Qh, Kh, sel_gpu, max_heads: int = 24):
+    """Routing of the timed run against the oracle (part of the oracle leg):
+    every row of up to ``max_heads`` heads, each classified as exact, or as a
+    near-tie swap the contract admits (the oracle's near-tie rule; every pick a
+    routing candidate of the query, same count, scores in order up to near
+    ties), or as inadmissible. Near-tie rows are those whose adjacent sorted
+    candidate scores (the k-th and (k+1)-th, or two selected ones) are within
+    the tie tolerance, whether or not the GPU's order differs there."""
+    import oracle
+
+    t0 = time.perf_counter()
+    heads = [(b, h) for b in range(wl.B) for h in range(wl.H)]
+    if len(heads) > max_heads:
+        step = len(heads) / max_heads
+        heads = [heads[int(i * step)] for i in range(max_heads)]
+    w1 = wl.replace(B=1, H=1)
+    lay = oracle.Layout(w1)
+    tot = {"exact": 0, "mismatch": 0, "near_tie_rows": 0, "inadmissible": 0}
+    first_bad = None
+    for b, h in heads:
+        q, kk = (t[b:b + 1, h:h + 1].contiguous() for t in (Qh, Kh))
+        kbar = oracle.pool(w1, kk, lay)
+        rt = oracle.route(w1, q, kbar, lay=lay)
+        res = oracle.check_selection(w1, q, kbar, np.ascontiguousarray(sel_gpu[b:b + 1, h:h + 1]), rt, lay)
+        for key in ("exact", "mismatch", "near_tie_rows"):
+            tot[key] += res[key]
+        tot["inadmissible"] += len(res["bad"])
+        if res["bad"] and first_bad is None:
+            first_bad = dict(res["bad"][0], b=b, h=h)
+    out = {"heads_checked": len(heads), "rows_checked": len(heads) * wl.L, **tot,
+           "rule": "near tie: adjacent sorted candidate scores within 1e-4 relative (or 1e-5 of "
+                   "sum |q_e Kbar_e|)", "seconds": round(time.perf_counter() - t0, 2)}
+    if first_bad is not None:
+        out["first_inadmissible"] = first_bad
+    return out
+
+
 def run_reference(args):
-    """Reference arm: the CPU oracle, timed on this host's cores, each step a
-    bounded sample of the same workload (rank 0 only)."""
+    """Reference arm: the CPU oracle, timed on this host's cores (rank 0 only).
+    Each step is a bounded sample of the same workload: routing and attention
+    of ``rows_per_step`` uniformly drawn query rows of head (0, 0), after the
+    head's pooling (done once, before the timed steps). ``value`` is the
+    sample's own throughput in whole-problem tokens (a token is one query row
+    of every head: rows / (B*H) tokens per step), so value * ms_per_step / 1e3
+    is the tokens one step processes; the time the oracle would need for the
+    whole scene is reported beside it."""
     ws_, rank, _ = dist_env()
     if rank != 0:
         return
@@ -446,33 +571,33 @@ def run_reference(args):
     lay = oracle.Layout(w1)
     rng = np.random.default_rng(1)
     rows_per_step = 48
-    t_pool = None
+    t0 = time.perf_counter()
+    kbar = oracle.pool(w1, kk, lay)
+    t_pool = time.perf_counter() - t0
     times = []
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        if t_pool is None:
-            kbar = oracle.pool(w1, kk, lay)
-            t_pool = time.perf_counter() - t0
-            t0 = time.perf_counter()
         rows = np.sort(rng.integers(0, lay.L, size=rows_per_step))
         rt = oracle.route(w1, q, kbar, rows=rows, lay=lay)
         oracle.attend(w1, q, kk, v, rt["sel"], rows=rows, lay=lay)
         if i >= args.warmup:
             times.append(time.perf_counter() - t0)
-    t_row = sum(times) / (len(times) * rows_per_step)
-    per_head = t_pool + t_row * lay.L
-    value = wl.B * wl.L / (per_head * wl.B * wl.H)
-    ms_per_step = per_head * wl.B * wl.H * 1e3
+    step_s = sum(times) / len(times)
+    tokens_per_step = rows_per_step / (wl.B * wl.H)
+    value = tokens_per_step / step_s
+    scene_s = (t_pool + step_s * lay.L / rows_per_step) * wl.B * wl.H
+    sample = (f"per step {rows_per_step} uniform query rows of head (0,0) (route + attend) = "
+              f"{tokens_per_step:.3f} tokens of the {wl.B}x{wl.H}-head problem; head pooling once "
+              f"before timing ({t_pool:.3f} s)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": ws_, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"{wl.name}: B={wl.B} H={wl.H} L={wl.L} d={wl.d} k={wl.k}"},
+            "config": {"workload": workload_string(wl, lay.C),
+                       "tokens_per_step": tokens_per_step},
+            "extrapolated_ms_per_scene": scene_s * 1e3,
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.threads(),
-                             "kind": "oracle",
-                             "sample": f"per step {rows_per_step} uniform query rows of head (0,0) "
-                                       f"(route + attend), pooling once ({t_pool:.2f} s); "
-                                       f"extrapolated to the whole scene"},
+                             "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -489,12 +614,17 @@ def main():
     ap.add_argument("--heads", type=int, default=None,
                     help="run the scene with this many heads instead (small profiling captures)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--shard", default="heads", choices=["heads", "replicas"],
+                    help="N > 1: split one scene's (b, h) slices over the ranks (strong scaling), "
+                         "or run an independent scene per rank (weak scaling)")
+    ap.add_argument("--gather", action="store_true",
+                    help="with --shard heads: all-gather the output slices after the timed steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense-compare", action="store_true",
                     help="skip the dense and FLOP-matched block-diagonal runs of the attention kernel")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
-        args.warmup = 3
+        ap.error("--warmup must be at least 3 (timing rule: three untimed steps before the timed ones)")
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -67,8 +67,10 @@ SIGNATURES = {
     "moc_attention_fwd": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _F, _P, _P, _P, _SZ, _P]),
     "moc_attention_fwd_static": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _F, _P, _P, _P]),
     "moc_check_device_error": (_I, [_P, _SZ, _P, _P]),
+    "moc_check_device_error_static": (_I, [_P, _P]),
     "moc_layout_device_error": (_I, [_P, _P, _P]),
     "moc_selftest_bounded_wait": (_I, [_P, _P]),
+    "moc_set_attend_schedule": (_I, [_I, _I]),
     "moc_forward_host": (_I, [_P, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _P, _P, _P, _SZ, _I, _P]),
     "moc_forward_host_device_bytes": (_SZ, [_P, _I, _I, _I, _I, _I]),
     "moc_route_perturb": (_I, [_P, _I, _I, _I, _I, _P, _P, _F, _F, _I, _P, _P]),
@@ -331,6 +333,12 @@ def check_layout_error(layout: Layout) -> int:
     _check(lib().moc_layout_device_error(layout.handle, ctypes.byref(det), _stream()),
            "layout device error word")
     return det.value
+
+
+def set_attend_schedule(n_ctas: int = 0, reverse: bool = False):
+    """Diagnostic: attention-kernel CTA count (0: one per SM) and item order for
+    the following calls (moc_set_attend_schedule)."""
+    _check(lib().moc_set_attend_schedule(int(n_ctas), 1 if reverse else 0), "moc_set_attend_schedule")
 
 
 def check_device_error(ws: torch.Tensor) -> int:

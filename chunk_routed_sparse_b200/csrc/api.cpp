@@ -1,6 +1,7 @@
 // C-ABI entry points: argument validation, workspace carve-up and kernel
 // launches. Every compute call is asynchronous on the caller's stream and
 // allocates nothing.
+#include <atomic>
 #include <cmath>
 #include <cstring>
 
@@ -31,7 +32,20 @@ moc_status check_common(const moc_layout* lay, int B, int H, int d, int k) {
 
 }  // namespace
 
+namespace {
+
+std::atomic<int> g_sched_ctas{0}, g_sched_reverse{0};
+
+}  // namespace
+
 namespace moc {
+
+AttendSchedule attend_schedule() {
+    AttendSchedule s;
+    s.n_ctas = g_sched_ctas.load(std::memory_order_relaxed);
+    s.reverse = g_sched_reverse.load(std::memory_order_relaxed);
+    return s;
+}
 
 WsPlan plan_workspace(const moc_layout* lay, int B, int H, int d, int k) {
     WsPlan p;
@@ -244,5 +258,12 @@ extern "C" moc_status moc_check_device_error(void* ws, size_t ws_bytes, int32_t*
     }
     if (h[0] == moc::ERR_TIMEOUT) return MOC_ERR_DEVICE_TIMEOUT;
     if (h[0] == moc::ERR_CHECK) return MOC_ERR_DEVICE_CHECK;
+    return MOC_OK;
+}
+
+extern "C" moc_status moc_set_attend_schedule(int n_ctas, int item_order) {
+    if (n_ctas < 0 || (item_order != 0 && item_order != 1)) return MOC_ERR_INVALID_ARG;
+    g_sched_ctas.store(n_ctas, std::memory_order_relaxed);
+    g_sched_reverse.store(item_order, std::memory_order_relaxed);
     return MOC_OK;
 }

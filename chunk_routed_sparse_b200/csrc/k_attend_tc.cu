@@ -174,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __nv_bfloat16* __restrict__ Q, int32_t* __restrict__ hdr,
                      const int32_t* __restrict__ qoff, const int32_t* __restrict__ tile_off,
                      const int32_t* __restrict__ qlist, float* __restrict__ lse_p,
-                     float* __restrict__ o_p) {
+                     float* __restrict__ o_p, int reverse) {
     using C = Cfg<D>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // 1024-byte aligned base: the 128-byte swizzle atoms of TMA and UMMA repeat every 1024 B
@@ -229,8 +229,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int it = 0;; ++it) {
                 const int slot = it & 1;
                 if (!wait_bar(bar(B_ITEM_EMPTY + slot), ((it >> 1) & 1) ^ 1, abort, hdr, 1)) break;
-                const int64_t item = atomicAdd(&hdr[HDR_WORK], 1);
-                const bool ok = item < total;
+                const int64_t ticket = atomicAdd(&hdr[HDR_WORK], 1);
+                const bool ok = ticket < total;
+                const int64_t item = reverse ? total - 1 - ticket : ticket;
                 sh.item[slot] = ok ? int(item) : -1;
                 mbar_arrive(bar(B_ITEM_FULL + slot));
                 if (!ok) break;
@@ -552,6 +553,8 @@ cudaError_t launch_d(const DevLayout& dv, int BH, const void* Q, const void* K, 
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const AttendSchedule sched = attend_schedule();
+    if (sched.n_ctas > 0 && sched.n_ctas < sms) sms = sched.n_ctas;
     int32_t* hdr = reinterpret_cast<int32_t*>(ws + p.hdr);
     e = cudaMemsetAsync(hdr + HDR_WORK, 0, sizeof(int32_t), s);
     if (e != cudaSuccess) return e;
@@ -559,7 +562,7 @@ cudaError_t launch_d(const DevLayout& dv, int BH, const void* Q, const void* K, 
         tmK, tmV, dv, BH, k, scale * 1.4426950408889634f, n_anchor, static_cast<const __nv_bfloat16*>(Q), hdr,
         reinterpret_cast<const int32_t*>(ws + p.qoff), reinterpret_cast<const int32_t*>(ws + p.tile_off),
         reinterpret_cast<const int32_t*>(ws + p.qlist), reinterpret_cast<float*>(ws + p.lse_p),
-        reinterpret_cast<float*>(ws + p.o_p));
+        reinterpret_cast<float*>(ws + p.o_p), sched.reverse);
     return cudaGetLastError();
 }
 

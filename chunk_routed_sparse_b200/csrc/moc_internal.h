@@ -78,6 +78,15 @@ WsPlan plan_workspace(const moc_layout* lay, int B, int H, int d, int k);
 enum { HDR_ERR = 0, HDR_DETAIL = 1, HDR_WORK = 2 };
 enum { ERR_NONE = 0, ERR_TIMEOUT = 1, ERR_CHECK = 2 };
 
+// Work schedule of the attention kernel (moc_set_attend_schedule): CTAs
+// (0: one per SM) and the order items are handed out in (reverse != 0: last
+// first). Results never depend on it.
+struct AttendSchedule {
+    int n_ctas = 0;
+    int reverse = 0;
+};
+AttendSchedule attend_schedule();
+
 // Kernel launchers (return cudaGetLastError() of the launch).
 cudaError_t launch_pool(const DevLayout& dv, int BH, int d, const void* K, float* Kbar,
                         cudaStream_t s);

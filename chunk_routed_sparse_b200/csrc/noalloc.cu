@@ -33,6 +33,24 @@ std::once_flag g_scratch_once[kMaxDevices];
 
 }  // namespace
 
+namespace {
+
+// The static scratch's device address on the current device (looked up once
+// per device, with that device current). Returns MOC_OK and sets *dev.
+moc_status static_scratch(void** ptr) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOC_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return MOC_ERR_UNSUPPORTED;
+    std::call_once(g_scratch_once[dev], [dev] {
+        g_scratch_err[dev] = cudaGetSymbolAddress(&g_scratch_dev[dev], g_static_scratch);
+    });
+    if (g_scratch_err[dev] != cudaSuccess || !g_scratch_dev[dev]) return MOC_ERR_CUDA;
+    *ptr = g_scratch_dev[dev];
+    return MOC_OK;
+}
+
+}  // namespace
+
 extern "C" moc_status moc_attention_fwd_static(const moc_layout* lay, int B, int H, int d,
                                                const void* Q, const void* K, const void* V,
                                                const int32_t* sel, int k, float softmax_scale,
@@ -43,13 +61,21 @@ extern "C" moc_status moc_attention_fwd_static(const moc_layout* lay, int B, int
     // the problem's scratch must fit the static area
     if (moc::plan_workspace(lay, B, H, d, k).total > kStaticScratchBytes)
         return MOC_ERR_WORKSPACE_TOO_SMALL;
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) return MOC_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return MOC_ERR_UNSUPPORTED;
-    std::call_once(g_scratch_once[dev], [dev] {
-        g_scratch_err[dev] = cudaGetSymbolAddress(&g_scratch_dev[dev], g_static_scratch);
-    });
-    if (g_scratch_err[dev] != cudaSuccess || !g_scratch_dev[dev]) return MOC_ERR_CUDA;
-    return moc_attention_fwd(lay, B, H, d, Q, K, V, sel, k, softmax_scale, O, lse,
-                             g_scratch_dev[dev], kStaticScratchBytes, stream);
+    void* scratch = nullptr;
+    const moc_status st = static_scratch(&scratch);
+    if (st != MOC_OK) return st;
+    return moc_attention_fwd(lay, B, H, d, Q, K, V, sel, k, softmax_scale, O, lse, scratch,
+                             kStaticScratchBytes, stream);
+}
+
+// The device error word of the calls above lives at the head of the static
+// scratch, whose address a caller cannot see; this reads and clears it on the
+// current device exactly as moc_check_device_error does for a caller workspace
+// (a later moc_attention_fwd_static call clears the word when it starts, so
+// check it after the call whose errors matter and before the next one).
+extern "C" moc_status moc_check_device_error_static(int32_t* detail, moc_stream_t stream) {
+    void* scratch = nullptr;
+    const moc_status st = static_scratch(&scratch);
+    if (st != MOC_OK) return st;
+    return moc_check_device_error(scratch, kStaticScratchBytes, detail, stream);
 }

@@ -189,12 +189,20 @@ moc_status moc_route_perturb(const moc_layout* layout, int B, int H, int k, int 
 /* Bytes of device workspace moc_attention_fwd and the three stage calls need
  * for this problem (0 on invalid arguments). Holds the per-chunk query lists,
  * the scheduler's counters and the partial outputs (1+k fp32 rows of d plus
- * a log-sum-exp per query). */
+ * a log-sum-exp per query): the storage of the attention over Omega(q) split
+ * into disjoint parts (Summary §3.1: Omega(q) is the union of the anchors and
+ * the selected chunks), which replaces the packed variable-length buffers of
+ * the jxzklqfsx.com write-up's "計算效率" section. */
 size_t moc_attention_workspace_bytes(const moc_layout* layout, int B, int H, int d, int k);
 
-/* (3) Query-list builder: invert sel into per-(b, h, chunk) lists of
- * (query, slot) entries by count -> exclusive prefix sum -> ordered scatter;
- * each list is sorted by query index. Fills the workspace. */
+/* (3) Query-list builder ("計算效率" of the jxzklqfsx.com write-up: the
+ * selected (query, chunk) pairs are grouped so that each chunk's keys are
+ * attended by all the queries that chose it, in place of its packing of
+ * variable-length groups for one FlashAttention varlen call): invert sel into
+ * per-(b, h, chunk) lists of (query, slot) entries by count -> exclusive
+ * prefix sum -> ordered scatter; each list is sorted by query index. Fills the
+ * workspace. An entry of sel that is >= C is ignored and recorded as
+ * MOC_ERR_DEVICE_CHECK (detail 3) in the workspace's error word. */
 moc_status moc_build_qlists(const moc_layout* layout, int B, int H, int k, const int32_t* sel,
                             void* ws, size_t ws_bytes, moc_stream_t stream);
 
@@ -209,14 +217,23 @@ moc_status moc_attend_partials(const moc_layout* layout, int B, int H, int d, co
                                const void* K, const void* V, int k, float softmax_scale,
                                void* ws, size_t ws_bytes, moc_stream_t stream);
 
-/* (5) Log-sum-exp merge of every query's partials: with M = max lse_j over the
- * valid slots, w_j = exp(lse_j - M), O = sum_j w_j O_j / sum_j w_j rounded to
- * bf16 (nearest even), lse = M + log sum_j w_j (fp32, nullable). Slots are
- * visited in a fixed order, so the result is deterministic. */
+/* (5) Log-sum-exp merge of every query's partials (Summary §3.1: softmax
+ * attention over Omega(q); Omega(q) is a disjoint union of the anchor keys and
+ * the selected chunks, and softmax over a disjoint union equals the
+ * log-sum-exp-weighted combination of the softmax over each part): with
+ * M = max lse_j over the valid slots, w_j = exp(lse_j - M),
+ * O = sum_j w_j O_j / sum_j w_j rounded to bf16 (nearest even),
+ * lse = M + log sum_j w_j (fp32, nullable). Slots are visited in a fixed order,
+ * so the result is deterministic. */
 moc_status moc_merge(const moc_layout* layout, int B, int H, int d, int k, const int32_t* sel,
                      void* O, float* lse, void* ws, size_t ws_bytes, moc_stream_t stream);
 
-/* Full attention stage: (3), (4) and (5) in order on one stream. */
+/* Full attention stage (Summary §3.1: o = Softmax(q K_Omega^T / sqrt(d))
+ * V_Omega over Omega(q) = anchors + the chunks in sel): (3), (4) and (5) in
+ * order on one stream. sel: device int32 [B][H][L][k] from (2) or (2'),
+ * -1 padded (NULL when k == 0); O: device bf16 [B][H][L][d]; lse: device fp32
+ * [B][H][L] (nullable); ws: the caller's workspace, 256-byte aligned, of at
+ * least moc_attention_workspace_bytes() bytes. */
 moc_status moc_attention_fwd(const moc_layout* layout, int B, int H, int d, const void* Q,
                              const void* K, const void* V, const int32_t* sel, int k,
                              float softmax_scale, void* O, float* lse, void* ws,
@@ -237,6 +254,14 @@ moc_status moc_attention_fwd(const moc_layout* layout, int B, int H, int d, cons
 moc_status moc_attention_fwd_static(const moc_layout* layout, int B, int H, int d, const void* Q,
                                     const void* K, const void* V, const int32_t* sel, int k,
                                     float softmax_scale, void* O, float* lse, moc_stream_t stream);
+
+/* Read and clear the device error word of moc_attention_fwd_static on the
+ * current device (its scratch, and so its error word, is not visible to the
+ * caller). The pages describe no counterpart. Synchronises the stream; returns
+ * what moc_check_device_error returns for a caller workspace. Every
+ * moc_attention_fwd_static call clears the word when it starts, so read it
+ * after the call whose errors matter and before the next one. */
+moc_status moc_check_device_error_static(int32_t* detail, moc_stream_t stream);
 
 /* Whole forward pass on HOST buffers: (1) pooling, (2) routing (when k > 0)
  * and (3)-(5) for every (b, h) slice, the end-to-end call for inputs that live
@@ -279,6 +304,15 @@ moc_status moc_check_device_error(void* ws, size_t ws_bytes, int32_t* detail,
  * moc_check_device_error then reports MOC_ERR_DEVICE_TIMEOUT) and returns;
  * nothing hangs or faults. Asynchronous on the stream. */
 moc_status moc_selftest_bounded_wait(int32_t* dev_word, moc_stream_t stream);
+
+/* Diagnostic (the pages have no counterpart): the work schedule of the
+ * attention kernel (4) for the calls that follow in this process - n_ctas
+ * persistent CTAs (0: one per SM; more than the SM count means one per SM)
+ * taking the work items in their natural order (item_order 0: anchor items,
+ * longest first, then routed items) or reversed (1). Every item is computed
+ * by one CTA from its inputs alone, so results do not depend on the schedule;
+ * tests use this to show it. Not thread-safe against concurrent launches. */
+moc_status moc_set_attend_schedule(int n_ctas, int item_order);
 
 /* Read and clear the device error word kept with a layout, where kernels that
  * run without a workspace (the router, (2)) record a bounded wait that gave up.

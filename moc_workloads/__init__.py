@@ -234,6 +234,31 @@ def make_qkv(wl: Workload, heads: Optional[Sequence[Tuple[int, int]]] = None, th
     return Q, K, V
 
 
+def make_qkv_slices(wl: Workload, s0: int, s1: int, threads: int = 8):
+    """Q, K, V of the flat (b, h) slices s0 .. s1-1 (slice i is b = i // H,
+    h = i % H) as bf16 CPU tensors [1, s1 - s0, L, d]: the same bytes those
+    slices have in ``make_qkv(wl)``, for a process that holds only a share of
+    the heads."""
+    n = s1 - s0
+    Q = torch.zeros(1, n, wl.L, wl.d, dtype=torch.bfloat16)
+    K = torch.zeros_like(Q)
+    V = torch.zeros_like(Q)
+
+    def one(i):
+        q, k, v = _gen_slice(wl, i // wl.H, i % wl.H)
+        Q[0, i - s0].copy_(q)
+        K[0, i - s0].copy_(k)
+        V[0, i - s0].copy_(v)
+
+    if threads > 1 and n > 1:
+        with ThreadPoolExecutor(max_workers=threads) as ex:
+            list(ex.map(one, range(s0, s1)))
+    else:
+        for i in range(s0, s1):
+            one(i)
+    return Q, K, V
+
+
 def bf16_bits(t: torch.Tensor) -> torch.Tensor:
     """View a bf16 tensor's storage as int16 (the raw bit patterns)."""
     assert t.dtype == torch.bfloat16

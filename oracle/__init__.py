@@ -196,6 +196,68 @@ def is_near(s1, s2, a1, a2):
            (gap < MAG_TIE * np.maximum(a1, a2))
 
 
+def check_selection(wl, Q: torch.Tensor, Kbar: np.ndarray, sel_other: np.ndarray, rt: dict,
+                    lay: Optional[Layout] = None) -> dict:
+    """Classify a selection computed elsewhere (in lower precision) against this
+    oracle's routing ``rt`` of the same rows (``route``): sel_other is
+    [B, H, nrows, k]. A row is exact when it equals the oracle's selection. A
+    differing row is admissible only when all of these hold:
+      - the oracle flags the row as near-tied (``near_tie_flags``);
+      - every pick is a routing candidate of the query's chunk (role CAND in the
+        oracle's own role table: never a mandatory or caption chunk, never a
+        chunk the causal mask hides), with no repeats and the same number of
+        -1 pads as the oracle;
+      - position by position, the pick's fp64 score equals or is near the
+        oracle's sorted score there, and the picks are in non-increasing score
+        order up to near ties.
+    Returns counts and the (b, h, r) indices of the mismatched and of the
+    inadmissible rows, with a reason for each inadmissible one."""
+    lay = lay or Layout(wl)
+    sel_o = rt["sel"]
+    k = sel_o.shape[-1]
+    out = {"rows": int(np.prod(sel_o.shape[:3])), "exact": 0, "mismatch": 0, "near_tie_rows": 0,
+           "mismatch_rows": [], "bad": []}
+    if k == 0:
+        out["exact"] = out["rows"]
+        return out
+    flags = near_tie_flags(rt)
+    near = flags["boundary"] | flags["inner"]
+    eq = np.all(sel_o == sel_other, axis=-1)
+    out["exact"] = int(eq.sum())
+    out["near_tie_rows"] = int(near.sum())
+    mism = [tuple(int(x) for x in m) for m in np.argwhere(~eq)]
+    out["mismatch"] = len(mism)
+    out["mismatch_rows"] = mism
+    for b, h, r in mism:
+        t = int(rt["rows"][r])
+        g, o = sel_other[b, h, r], sel_o[b, h, r]
+        gv = g[g >= 0]
+        why = None
+        if not near[b, h, r]:
+            why = "no near tie"
+        elif (g < 0).sum() != (o < 0).sum():
+            why = "different number of picks"
+        elif len(set(gv.tolist())) != len(gv):
+            why = "repeated pick"
+        elif np.any(gv >= lay.C) or np.any(lay.role[lay.chunk_of_token[t], gv] != ROLE_CAND):
+            why = "pick is not a routing candidate of the query"
+        else:
+            bh = b * wl.H + h
+            s, a = scores(wl, Q, Kbar, [bh] * len(gv), [t] * len(gv), gv, lay)
+            so, ao = rt["top_s"][b, h, r, :len(gv)], rt["top_a"][b, h, r, :len(gv)]
+            for x in range(len(gv)):
+                if not (s[x] == so[x] or is_near(s[x], so[x], a[x], ao[x])):
+                    why = f"score at position {x} not near the oracle's"
+                    break
+                if x + 1 < len(gv) and not (s[x] >= s[x + 1] or is_near(s[x], s[x + 1], a[x], a[x + 1])):
+                    why = f"positions {x}, {x + 1} out of order"
+                    break
+        if why is not None:
+            out["bad"].append({"b": b, "h": h, "row": t, "why": why, "sel": g.tolist(),
+                               "oracle": o.tolist()})
+    return out
+
+
 def near_tie_flags(rt: dict) -> dict:
     """Per row: 'boundary' = k-th and (k+1)-th candidates near-tied;
     'inner' = two adjacent selected entries near-tied (their order may swap)."""

@@ -57,3 +57,45 @@ def test_reference_arm_under_torchrun_prints_once():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_head_split_covers_every_slice_once_and_balanced():
+    import bench
+    for B, H in [(1, 24), (2, 24), (1, 5), (3, 7)]:
+        for world in (1, 2, 3, 4, 8):
+            shares = [bench.shard_slices(B, H, world, r) for r in range(world)]
+            covered = [i for a, b in shares for i in range(a, b)]
+            assert covered == list(range(B * H)), (B, H, world)
+            sizes = [b - a for a, b in shares]
+            assert max(sizes) - min(sizes) <= 1
+
+
+def _gather_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    sys.path.insert(0, ROOT)
+    import bench
+    import moc_workloads as W
+    wl = W.tiny().replace(B=2, H=3)            # 6 slices over `world` ranks
+    s0, s1 = bench.shard_slices(wl.B, wl.H, world, rank)
+    q, _, _ = W.make_qkv_slices(wl, s0, s1)    # this rank's share of the scene's Q
+    full = bench.gather_slices(q.view(s1 - s0, wl.L, wl.d), wl.B * wl.H, world)
+    out[rank] = full.view(torch.int16).numpy().tobytes()
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_head_split_shares_reassemble_the_whole_tensor(world):
+    """Each rank generates only its slices; the all-gather of the shares must
+    equal the whole tensor built by one process on the CPU."""
+    import moc_workloads as W
+    wl = W.tiny().replace(B=2, H=3)
+    ref, _, _ = W.make_qkv(wl)
+    port = _free_port()
+    with mp.get_context("spawn").Manager() as m:
+        out = m.dict()
+        mp.start_processes(_gather_worker, args=(world, port, out), nprocs=world, start_method="spawn")
+        got = [out[r] for r in range(world)]
+    want = ref.view(wl.B * wl.H, wl.L, wl.d).view(torch.int16).numpy().tobytes()
+    assert all(g == want for g in got)

@@ -84,7 +84,7 @@ def test_attention_over_a_perturbed_selection():
     O, lse = moc.attention_fwd(lay, Q.cuda(), K.cuda(), V.cuda(), torch.from_numpy(out).cuda(), k + m_max)
     torch.cuda.synchronize()
     O_o, lse_o, _ = oracle.attend(wl, Q, K, V, ref, rows=rows, lay=orc)
-    compare_attention(O.cpu(), lse.cpu(), O_o, lse_o, np.ones(O_o.shape[:3], dtype=bool))
+    compare_attention(O.cpu(), lse.cpu(), O_o, lse_o)
 
 
 def test_argument_checks():
