@@ -1,7 +1,10 @@
 """Benchmark of the MoC sparse-attention forward pass (one JSON line on rank 0).
 
 A step is one pass of the whole hot path over one scene: (1) pool keys,
-(2) route, (3) build query lists, (4) attend, (5) merge. Default workload:
+(2) route, (3) build query lists, (4) attend with (5) the log-sum-exp merge
+fused into it (moc_attend_merged, the path moc_attention_fwd takes). The
+unfused stage calls - (4) writing every partial, then (5) as its own kernel -
+are timed once after the steps for the per-kernel roofline of (5). Default workload:
 the eight-shot 180,512-token scene (B=1, H=24, d=128, k=3). Inputs are larger
 than L2 (3 x 1.1 GB), so no L2 flush is needed between steps.
 
@@ -38,8 +41,8 @@ sys.path.insert(0, ROOT)
 import moc_workloads as W  # noqa: E402
 
 METRIC = "MoC fwd tokens/s and selected-pair TFLOP/s (% bf16 peak) at 180k tokens"
-STAGES = ["pool", "route", "qlist", "attend", "merge"]
-LAUNCHES_PER_STEP = {"pool": 1, "route": 1, "qlist": 4, "attend": 1, "merge": 1}
+STAGES = ["pool", "route", "qlist", "attend"]  # attend = (4) with the merge (5) fused in
+LAUNCHES_PER_STEP = {"pool": 1, "route": 1, "qlist": 4, "attend": 1}
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -259,10 +262,8 @@ def run_ours(args):
         if ev: ev[2].record(stream)
         moc.build_qlists(lay, sel, B, H, k, ws)
         if ev: ev[3].record(stream)
-        moc.attend_partials(lay, Q, K, V, k, ws, scale)
+        moc.attend_merged(lay, Q, K, V, sel, k, ws, O, lse, scale)
         if ev: ev[4].record(stream)
-        moc.merge(lay, sel, k, ws, O, lse)
-        if ev: ev[5].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -275,7 +276,7 @@ def run_ours(args):
         if ws_ > 1:
             torch.distributed.barrier()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(args.steps)]
     clocks = ClockSampler(local)
     barrier()
     torch.cuda.synchronize()
@@ -293,6 +294,7 @@ def run_ours(args):
     stage_ms = {s: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
                 for j, s in enumerate(STAGES)}
     moc.check_device_error(ws)
+    unfused = unfused_timing(moc, lay, Q, K, V, sel, k, ws, scale, stream, B, H, L, d)
 
     # end to end through the C ABI's host-buffer call (moc_forward_host): pinned host
     # Q, K, V in, host O back; inside, chunks of heads are uploaded, computed and
@@ -375,17 +377,22 @@ def run_ours(args):
                      "peak_kind": f"bf16_tflops_sustained ({peak_src})",
                      "frac_of_burst": achieved_tf / float(peaks.get("bf16_tflops", 1590.0)),
                      "traffic": traffic},
-        "hbm_kernels": hbm_fracs(stage_ms, B, H, L, lay.C, d, k, peaks, routed_rows(lay, wl),
-                                 int((sel >= 0).sum().item()) if k > 0 else 0),
+        "hbm_kernels": hbm_fracs(dict(stage_ms, merge=unfused["merge_ms"]), B, H, L, lay.C, d, k, peaks,
+                                 routed_rows(lay, wl), int((sel >= 0).sum().item()) if k > 0 else 0),
+        "unfused_stage_calls": unfused,
         "clocks": clk,
         "e2e": {"value": job_tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                 "ms_per_step": e2e_ms,
                 "path": "moc_forward_host: host buffers, 12 chunks of heads, copies overlapped",
                 "h2d_bytes_per_step": 3 * Q.numel() * 2, "d2h_bytes_per_step": O.numel() * 2},
         "gpu_launches": args.steps * sum(LAUNCHES_PER_STEP.values()),
+        "gpu_launches_breakdown": {"per_step": LAUNCHES_PER_STEP,
+                                   "note": "kernels of this library in the device-timed steps"},
     }
     if gather is not None:
         line["gather"] = gather
+    if not args.no_backward:
+        line["backward"] = backward_timing(moc, lay, Q, K, V, O, lse, sel, k, pairs, d, stream)
     if ws_ == 1 and not args.no_dense_compare and wl.name == "eight":
         line["dense_compare"] = dense_compare(moc, wl, Q, K, V, O, lse, stream, pairs,
                                               stage_ms, ms_per_step, peak_tf)
@@ -446,11 +453,65 @@ def dense_compare(moc, wl, Q, K, V, O, lse, stream, moc_pairs, stage_ms, moc_ste
                      "tflops": 4.0 * d * pairs / (a / 1e3) / 1e12,
                      "frac_sustained": 4.0 * d * pairs / (a / 1e3) / 1e12 / peak_tf}
         del ws
-    moc_attention_ms = stage_ms["qlist"] + stage_ms["attend"] + stage_ms["merge"]
+    moc_attention_ms = stage_ms["qlist"] + stage_ms["attend"]
     out["moc_pairs"] = moc_pairs
     out["moc_step_speedup_vs_dense"] = out["dense"]["step_ms"] / moc_step_ms
     out["moc_attention_vs_flop_matched"] = moc_attention_ms / out["flop_matched"]["attention_ms"]
     return out
+
+
+def unfused_timing(moc, lay, Q, K, V, sel, k, ws, scale, stream, B, H, L, d, reps=3):
+    """The stage calls of the unfused path after the timed steps: (4) writing
+    every partial (moc_attend_partials), then (5) as its own kernel (moc_merge);
+    mean of ``reps`` after one untimed run."""
+    O2 = torch.empty_like(Q)
+    lse2 = torch.empty(B, H, L, dtype=torch.float32, device=Q.device)
+    att, mer = [], []
+    for it in range(1 + reps):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        moc.build_qlists(lay, sel, B, H, k, ws)
+        ev[0].record(stream)
+        moc.attend_partials(lay, Q, K, V, k, ws, scale)
+        ev[1].record(stream)
+        moc.merge(lay, sel, k, ws, O2, lse2)
+        ev[2].record(stream)
+        torch.cuda.synchronize()
+        if it >= 1:
+            att.append(ev[0].elapsed_time(ev[1]))
+            mer.append(ev[1].elapsed_time(ev[2]))
+    moc.check_device_error(ws)
+    del O2, lse2
+    return {"attend_partials_ms": statistics.mean(att), "merge_ms": statistics.mean(mer)}
+
+
+def backward_timing(moc, lay, Q, K, V, O, lse, sel, k, pairs, d, stream, reps=5):
+    """The backward pass (moc_attention_bwd: query lists, D = dO . o, the dQ
+    kernel, the dQ reduce, the dK / dV kernel) for a seeded upstream gradient,
+    over the forward pass's selection and outputs; CUDA events around each
+    call after 2 untimed calls, mean of ``reps``. Selected-pair FLOPs follow the
+    usual 2.5x-forward count (10 d per kept pair: S, dP, dV, dK, dQ); the
+    kernels execute 14 d (S and dP are formed once per side)."""
+    B, H, L, _ = Q.shape
+    g = torch.Generator(device=Q.device).manual_seed(99)
+    dO = torch.randn(Q.shape, device=Q.device, generator=g).to(torch.bfloat16)
+    n = int(moc.lib().moc_attention_bwd_workspace_bytes(lay.handle, B, H, d, k))
+    ws = torch.empty(n, dtype=torch.uint8, device=Q.device)
+    dQ, dK, dV = torch.empty_like(Q), torch.empty_like(Q), torch.empty_like(Q)
+    ts = []
+    for it in range(2 + reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        moc.attention_bwd(lay, Q, K, V, O, lse, dO, sel, k, ws=ws, dQ=dQ, dK=dK, dV=dV)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if it >= 2:
+            ts.append(e0.elapsed_time(e1))
+    moc.check_device_error(ws)
+    ms = statistics.mean(ts)
+    del ws, dO, dQ, dK, dV
+    return {"ms": ms, "tflops_selected_pairs_10d": 10.0 * d * pairs / (ms / 1e3) / 1e12,
+            "tflops_executed_14d": 14.0 * d * pairs / (ms / 1e3) / 1e12,
+            "launches": 4 + 4, "workspace_bytes": n}
 
 
 def routed_rows(lay, wl) -> int:
@@ -614,6 +675,8 @@ def main():
     ap.add_argument("--heads", type=int, default=None,
                     help="run the scene with this many heads instead (small profiling captures)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the timing of the backward pass (moc_attention_bwd) after the forward steps")
     ap.add_argument("--shard", default="heads", choices=["heads", "replicas"],
                     help="N > 1: split one scene's (b, h) slices over the ranks (strong scaling), "
                          "or run an independent scene per rank (weak scaling)")

@@ -64,8 +64,12 @@ SIGNATURES = {
     "moc_build_qlists": (_I, [_P, _I, _I, _I, _P, _P, _SZ, _P]),
     "moc_attend_partials": (_I, [_P, _I, _I, _I, _P, _P, _P, _I, _F, _P, _SZ, _P]),
     "moc_merge": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _SZ, _P]),
+    "moc_attend_merged": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _F, _P, _P, _P, _SZ, _P]),
     "moc_attention_fwd": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _F, _P, _P, _P, _SZ, _P]),
     "moc_attention_fwd_static": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _F, _P, _P, _P]),
+    "moc_attention_bwd_workspace_bytes": (_SZ, [_P, _I, _I, _I, _I]),
+    "moc_attention_bwd": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _I, _F, _P, _P, _P, _P, _SZ,
+                               _P]),
     "moc_check_device_error": (_I, [_P, _SZ, _P, _P]),
     "moc_check_device_error_static": (_I, [_P, _P]),
     "moc_layout_device_error": (_I, [_P, _P, _P]),
@@ -256,6 +260,15 @@ def attend_partials(layout, Q, K, V, k, ws, scale=None):
            "moc_attend_partials")
 
 
+def attend_merged(layout, Q, K, V, sel, k, ws, O, lse=None, scale=None):
+    """(4) + (5) fused (moc_attend_merged); needs build_qlists first."""
+    B, H, L, d = _dims(Q)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    _check(lib().moc_attend_merged(layout.handle, B, H, d, _ptr(Q), _ptr(K), _ptr(V),
+                                   _ptr(sel) if k > 0 else None, k, float(scale), _ptr(O), _ptr(lse),
+                                   _ptr(ws), ws.numel(), _stream()), "moc_attend_merged")
+
+
 def merge(layout, sel, k, ws, O, lse=None):
     B, H, L, d = _dims(O)
     _check(lib().moc_merge(layout.handle, B, H, d, k, _ptr(sel) if k > 0 else None, _ptr(O),
@@ -281,6 +294,33 @@ def attention_fwd(layout: Layout, Q, K, V, sel, k: int, scale: Optional[float] =
                                    _ptr(lse), _ptr(ws), ws.numel(), _stream()),
            "moc_attention_fwd")
     return O, lse
+
+
+def attention_bwd(layout: Layout, Q, K, V, O, lse, dO, sel, k: int, scale: Optional[float] = None,
+                  ws: Optional[torch.Tensor] = None, dQ: Optional[torch.Tensor] = None,
+                  dK: Optional[torch.Tensor] = None, dV: Optional[torch.Tensor] = None):
+    """Backward of attention_fwd (moc_attention_bwd): returns bf16 (dQ, dK, dV)
+    for the upstream gradient dO, with the selection held constant."""
+    B, H, L, d = _dims(Q)
+    for t in (K, V, O, dO):
+        if tuple(t.shape) != (B, H, L, d) or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("Q, K, V, O, dO must be contiguous bf16 [B, H, L, d] tensors")
+    if tuple(lse.shape) != (B, H, L) or lse.dtype != torch.float32:
+        raise ValueError("lse must be fp32 [B, H, L]")
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if ws is None:
+        n = int(lib().moc_attention_bwd_workspace_bytes(layout.handle, B, H, d, k))
+        if n == 0:
+            raise ValueError("invalid problem for the backward workspace size query")
+        ws = torch.empty(n, dtype=torch.uint8, device=Q.device)
+    dQ = torch.empty_like(Q) if dQ is None else dQ
+    dK = torch.empty_like(Q) if dK is None else dK
+    dV = torch.empty_like(Q) if dV is None else dV
+    _check(lib().moc_attention_bwd(layout.handle, B, H, d, _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse),
+                                   _ptr(dO), _ptr(sel) if k > 0 else None, k, float(scale), _ptr(dQ),
+                                   _ptr(dK), _ptr(dV), _ptr(ws), ws.numel(), _stream()),
+           "moc_attention_bwd")
+    return dQ, dK, dV
 
 
 def forward(layout: Layout, Q, K, V, k: int, causal: bool = True, scale=None, ws=None):

@@ -68,6 +68,18 @@ WsPlan plan_workspace(const moc_layout* lay, int B, int H, int d, int k) {
     return p;
 }
 
+WsPlan plan_workspace_bwd(const moc_layout* lay, int B, int H, int d, int k) {
+    WsPlan p = plan_workspace(lay, B, H, d, k);
+    const size_t BH = size_t(B) * H, L = size_t(lay->L), S = size_t(k) + 1;
+    size_t off = p.lse_p;
+    p.lse_p = off;  // D = dO . o per row
+    off += align256(BH * L * sizeof(float));
+    p.o_p = off;    // dQ partial rows
+    off += align256(BH * L * S * size_t(d) * sizeof(float));
+    p.total = off;
+    return p;
+}
+
 }  // namespace moc
 
 extern "C" const char* moc_status_string(moc_status s) {
@@ -103,7 +115,8 @@ extern "C" moc_status moc_route(const moc_layout* lay, int B, int H, int d, cons
         (reinterpret_cast<uintptr_t>(sel) & 3))
         return MOC_ERR_INVALID_ARG;
     return cuda_status(moc::launch_route(lay->dv, B * H, lay->total_rtiles, d, Q, Kbar, k,
-                                         causal ? 1 : 0, nullptr, sel, (cudaStream_t)stream));
+                                         causal ? 1 : 0, lay->max_cand, nullptr, sel,
+                                         (cudaStream_t)stream));
 }
 
 extern "C" moc_status moc_outer_route(const moc_layout* lay, int B, int H, int d, const float* Qbar,
@@ -132,7 +145,8 @@ extern "C" moc_status moc_route_masked(const moc_layout* lay, int B, int H, int 
         (reinterpret_cast<uintptr_t>(sel) & 3) || (reinterpret_cast<uintptr_t>(seg_mask) & 7))
         return MOC_ERR_INVALID_ARG;
     return cuda_status(moc::launch_route(lay->dv, B * H, lay->total_rtiles, d, Q, Kbar, k,
-                                         causal ? 1 : 0, seg_mask, sel, (cudaStream_t)stream));
+                                         causal ? 1 : 0, lay->max_cand, seg_mask, sel,
+                                         (cudaStream_t)stream));
 }
 
 extern "C" moc_status moc_route_perturb(const moc_layout* lay, int B, int H, int k, int causal,
@@ -210,6 +224,24 @@ extern "C" moc_status moc_attend_partials(const moc_layout* lay, int B, int H, i
                                              static_cast<char*>(ws), p, (cudaStream_t)stream));
 }
 
+extern "C" moc_status moc_attend_merged(const moc_layout* lay, int B, int H, int d, const void* Q,
+                                        const void* K, const void* V, const int32_t* sel, int k, float scale,
+                                        void* O, float* lse, void* ws, size_t ws_bytes, moc_stream_t stream) {
+    moc_status st = check_common(lay, B, H, d, k);
+    if (st != MOC_OK) return st;
+    if (B * H == 0) return MOC_OK;
+    moc::WsPlan p;
+    if ((st = check_ws(lay, B, H, d, k, ws, ws_bytes, &p)) != MOC_OK) return st;
+    if (!Q || !K || !V || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+        return MOC_ERR_INVALID_ARG;
+    if (k > 0 && (!sel || (reinterpret_cast<uintptr_t>(sel) & 3))) return MOC_ERR_INVALID_ARG;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3)) return MOC_ERR_INVALID_ARG;
+    if (!(scale > 0.0f) || scale != scale) return MOC_ERR_INVALID_ARG;
+    const int64_t n_anchor = int64_t(B) * H * lay->total_atiles;
+    return cuda_status(moc::launch_attend_merged(lay->dv, B * H, d, Q, K, V, k, scale, n_anchor,
+                                                 static_cast<char*>(ws), p, sel, O, lse, (cudaStream_t)stream));
+}
+
 extern "C" moc_status moc_merge(const moc_layout* lay, int B, int H, int d, int k,
                                 const int32_t* sel, void* O, float* lse, void* ws, size_t ws_bytes,
                                 moc_stream_t stream) {
@@ -239,9 +271,7 @@ extern "C" moc_status moc_attention_fwd(const moc_layout* lay, int B, int H, int
     if (lse && (reinterpret_cast<uintptr_t>(lse) & 3)) return MOC_ERR_INVALID_ARG;
     if (!(scale > 0.0f) || scale != scale) return MOC_ERR_INVALID_ARG;
     if ((st = moc_build_qlists(lay, B, H, k, sel, ws, ws_bytes, stream)) != MOC_OK) return st;
-    if ((st = moc_attend_partials(lay, B, H, d, Q, K, V, k, scale, ws, ws_bytes, stream)) != MOC_OK)
-        return st;
-    return moc_merge(lay, B, H, d, k, sel, O, lse, ws, ws_bytes, stream);
+    return moc_attend_merged(lay, B, H, d, Q, K, V, sel, k, scale, O, lse, ws, ws_bytes, stream);
 }
 
 extern "C" moc_status moc_check_device_error(void* ws, size_t ws_bytes, int32_t* detail,
@@ -266,4 +296,38 @@ extern "C" moc_status moc_set_attend_schedule(int n_ctas, int item_order) {
     g_sched_ctas.store(n_ctas, std::memory_order_relaxed);
     g_sched_reverse.store(item_order, std::memory_order_relaxed);
     return MOC_OK;
+}
+
+extern "C" size_t moc_attention_bwd_workspace_bytes(const moc_layout* lay, int B, int H, int d, int k) {
+    if (!lay || B < 0 || H < 0 || (d != 64 && d != 128) || k < 0 || k > moc::kMaxK) return 0;
+    return moc::plan_workspace_bwd(lay, B, H, d, k).total;
+}
+
+extern "C" moc_status moc_attention_bwd(const moc_layout* lay, int B, int H, int d, const void* Q,
+                                        const void* K, const void* V, const void* O, const float* lse,
+                                        const void* dO, const int32_t* sel, int k, float scale, void* dQ,
+                                        void* dK, void* dV, void* ws, size_t ws_bytes, moc_stream_t stream) {
+    moc_status st = check_common(lay, B, H, d, k);
+    if (st != MOC_OK) return st;
+    if (B * H == 0) return MOC_OK;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return MOC_ERR_INVALID_ARG;
+    const moc::WsPlan p = moc::plan_workspace_bwd(lay, B, H, d, k);
+    if (ws_bytes < p.total) return MOC_ERR_WORKSPACE_TOO_SMALL;
+    for (const void* t : {Q, K, V, O, dO, static_cast<const void*>(dQ), static_cast<const void*>(dK),
+                          static_cast<const void*>(dV)})
+        if (!t || !aligned16(t)) return MOC_ERR_INVALID_ARG;
+    if (!lse || (reinterpret_cast<uintptr_t>(lse) & 3)) return MOC_ERR_INVALID_ARG;
+    if (k > 0 && (!sel || (reinterpret_cast<uintptr_t>(sel) & 3))) return MOC_ERR_INVALID_ARG;
+    if (!(scale > 0.0f) || scale != scale) return MOC_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    char* w = static_cast<char*>(ws);
+    const int BH = B * H;
+    cudaError_t e = moc::launch_qlists(lay->dv, BH, k, sel, w, p, s);
+    if (e == cudaSuccess) e = moc::launch_bwd_rowdot(BH, int(lay->L), d, O, dO, w, p, s);
+    if (e == cudaSuccess)
+        e = moc::launch_bwd_dq(lay->dv, BH, d, Q, K, V, dO, lse, k, scale, int64_t(BH) * lay->total_atiles, w, p,
+                               s);
+    if (e == cudaSuccess) e = moc::launch_bwd_dq_reduce(BH, int(lay->L), lay->C, d, k, sel, dQ, w, p, s);
+    if (e == cudaSuccess) e = moc::launch_bwd_dkv(lay->dv, BH, d, Q, K, V, dO, lse, scale, w, p, dK, dV, s);
+    return cuda_status(e);
 }

@@ -68,6 +68,12 @@ __device__ __forceinline__ bool ranks_before(float sa, int ja, float sb, int jb)
     return sa > sb || (sa == sb && ja < jb);
 }
 
+__device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t* p) {
+    int32_t v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ void set_error(int32_t* hdr, int code, int detail) {
     if (atomicCAS(&hdr[HDR_ERR], ERR_NONE, code) == ERR_NONE) atomicExch(&hdr[HDR_DETAIL], detail);
 }

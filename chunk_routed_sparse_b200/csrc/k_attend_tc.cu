@@ -41,6 +41,7 @@
 // Every mbarrier wait is bounded (2 s): on timeout the kernel records
 // ERR_TIMEOUT and a site code in the workspace header, every role leaves its
 // loop, in-flight copies and MMAs are drained (bounded) and TMEM is freed.
+#include "items.cuh"
 #include "pipeline.cuh"
 #include "tmap.cuh"
 
@@ -48,8 +49,12 @@ namespace moc {
 namespace {
 
 using namespace sm100;
+using items::Item;
+using items::Cursor;
+using items::decode;
+using items::count_tiles;
 
-constexpr int kKT = 128;                        // keys per tile
+using items::kKT;                               // keys per tile
 constexpr int kThreads = 384;                   // softmax A, softmax B, producer/MMA warpgroups
 // Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64512);
 // the producer/MMA warpgroup drops to 72 and the softmax warpgroups rise to
@@ -91,90 +96,20 @@ struct Shared {  // at oBar + 192
     int abort;
 };
 
-struct Item {
-    int bh, nq, slot_fixed, q0;
-    const int32_t* entries;
-    int r_beg, r_end, k0, k1;
-};
-
-__device__ __forceinline__ bool decode(const DevLayout& dv, int BH, int64_t n_anchor, int64_t item,
-                                       const int32_t* tile_off, const int32_t* qoff,
-                                       const int32_t* qlist, Item& it) {
-    if (item < n_anchor) {
-        const int pos = upper_index(dv.atile_off, dv.G + 1, item / BH);
-        const int64_t local = item - int64_t(BH) * dv.atile_off[pos];
-        const int nt = dv.atile_off[pos + 1] - dv.atile_off[pos];
-        const int g = dv.a_order[pos];
-        it.bh = int(local / nt);
-        it.q0 = dv.grp_q0[g] + int(local % nt) * kItemRows;
-        it.nq = min(kItemRows, dv.grp_q1[g] - it.q0);
-        it.slot_fixed = 0;
-        it.entries = nullptr;
-        it.r_beg = dv.ar_off[g];
-        it.r_end = dv.ar_off[g + 1];
-        it.k0 = it.k1 = 0;
-        return true;
-    }
-    const int64_t r = item - n_anchor;
-    const int64_t nlists = int64_t(BH) * dv.C;
-    if (r >= tile_off[nlists]) return false;
-    const int x = upper_index(tile_off, int(nlists + 1), r);
-    const int c = x % dv.C;
-    it.bh = x / dv.C;
-    const int e0 = qoff[x] + int(r - tile_off[x]) * kItemRows;
-    it.nq = min(kItemRows, qoff[x + 1] - e0);
-    it.entries = qlist + e0;
-    it.slot_fixed = -1;
-    it.q0 = 0;
-    it.r_beg = it.r_end = -1;
-    it.k0 = dv.chunk_off[c];
-    it.k1 = dv.chunk_off[c + 1];
-    return true;
-}
-
-// Key tiles of an item, in order: each range cut into 128-key tiles.
-struct Cursor {
-    const int32_t* ar;
-    int r, r_end, pos, end;
-    __device__ void init(const DevLayout& dv, const Item& it) {
-        if (it.r_beg >= 0) {
-            ar = dv.ar; r = it.r_beg; r_end = it.r_end;
-            pos = ar[2 * r];
-            end = ar[2 * r + 1];
-        } else {
-            ar = nullptr; r = 0; r_end = 1; pos = it.k0; end = it.k1;
-        }
-    }
-    __device__ bool more() const { return r < r_end; }
-    __device__ void next(int& key0, int& nvalid) {
-        key0 = pos;
-        nvalid = min(kKT, end - pos);
-        pos += kKT;
-        if (pos >= end) {
-            ++r;
-            if (ar && r < r_end) {
-                pos = ar[2 * r];
-                end = ar[2 * r + 1];
-            }
-        }
-    }
-};
-
-__device__ __forceinline__ int count_tiles(const DevLayout& dv, const Item& it) {
-    if (it.r_beg < 0) return (it.k1 - it.k0 + kKT - 1) / kKT;
-    int t = 0;
-    for (int r = it.r_beg; r < it.r_end; ++r) t += (dv.ar[2 * r + 1] - dv.ar[2 * r] + kKT - 1) / kKT;
-    return t;
-}
-
-template <int D>
+// FUSED: routed items run first and write their partials; every anchor item
+// then merges its own part with the routed partials of its rows in the epilogue
+// and writes the bf16 output row and its log-sum-exp (the merge of (5) done in
+// place, so slot 0 is never written and read back). Not FUSED: every item writes
+// its partial, for the stage call of (4) followed by (5).
+template <int D, bool FUSED>
 __global__ void __launch_bounds__(kThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      DevLayout dv, int BH, int k, float scale_log2, int64_t n_anchor,
                      const __nv_bfloat16* __restrict__ Q, int32_t* __restrict__ hdr,
                      const int32_t* __restrict__ qoff, const int32_t* __restrict__ tile_off,
                      const int32_t* __restrict__ qlist, float* __restrict__ lse_p,
-                     float* __restrict__ o_p, int reverse) {
+                     float* __restrict__ o_p, int reverse, const int32_t* __restrict__ sel,
+                     __nv_bfloat16* __restrict__ O_out, float* __restrict__ lse_out) {
     using C = Cfg<D>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // 1024-byte aligned base: the 128-byte swizzle atoms of TMA and UMMA repeat every 1024 B
@@ -231,7 +166,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!wait_bar(bar(B_ITEM_EMPTY + slot), ((it >> 1) & 1) ^ 1, abort, hdr, 1)) break;
                 const int64_t ticket = atomicAdd(&hdr[HDR_WORK], 1);
                 const bool ok = ticket < total;
-                const int64_t item = reverse ? total - 1 - ticket : ticket;
+                int64_t item = reverse ? total - 1 - ticket : ticket;
+                if (FUSED) {  // routed items first (each class in natural or reversed order)
+                    const int64_t n_routed = total - n_anchor;
+                    if (ticket < n_routed) item = n_anchor + (reverse ? n_routed - 1 - ticket : ticket);
+                    else item = reverse ? total - 1 - ticket : ticket - n_routed;
+                }
                 sh.item[slot] = ok ? int(item) : -1;
                 mbar_arrive(bar(B_ITEM_FULL + slot));
                 if (!ok) break;
@@ -492,6 +432,73 @@ __global__ void __launch_bounds__(kThreads, 1)
             // as whole 128-byte row pieces, four rows per store instruction.
             if (!wait_bar_warp(bar(B_PV_DONE + q), (gtt - 1) & 1, abort, hdr, 14)) break;
             tc_fence_after();
+            if (FUSED && itm.slot_fixed == 0) {
+                // merged epilogue of an anchor item: every routed row of this launch
+                // is complete once the counter of written routed rows reaches the
+                // number of query-list entries (routed items are handed out before
+                // any anchor item, so none of them waits behind this one)
+                if (lane == 0) {
+                    const int32_t target = qoff[int64_t(BH) * dv.C];
+                    const uint64_t t0 = globaltimer();
+                    while (ld_acquire_gpu(&hdr[HDR_RDONE]) < target) {
+                        if (globaltimer() - t0 > kTimeoutNs) { set_error(hdr, ERR_TIMEOUT, 16); break; }
+                    }
+                }
+                __syncwarp();
+                __threadfence();
+                const size_t row = size_t(itm.bh) * L + (my_tok >= 0 ? my_tok : 0);
+                const float lse0 = (m_used + log2f(l)) * 0.69314718055994531f;
+                // slots in fixed order: the own part (slot 0), then sel order
+                float M = lse0;
+                if (my_tok >= 0) {
+                    for (int x = 0; x < k; ++x) {
+                        const int32_t sj = sel[row * k + x];
+                        if (sj >= 0 && sj < dv.C) M = fmaxf(M, lse_p[row * S + 1 + x]);
+                    }
+                }
+                float Z = expf(lse0 - M);
+                if (my_tok >= 0) {
+                    for (int x = 0; x < k; ++x) {
+                        const int32_t sj = sel[row * k + x];
+                        if (sj >= 0 && sj < dv.C) Z += expf(lse_p[row * S + 1 + x] - M);
+                    }
+                }
+                const float a0 = expf(lse0 - M) / (Z * l);  // the own part is O / l
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(o_addr + c * 32, o);
+                    tmem_wait_ld_regs(o);
+                    float acc[32];
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) acc[x] = __uint_as_float(o[x]) * a0;
+                    if (my_tok >= 0) {
+                        for (int x = 0; x < k; ++x) {
+                            const int32_t sj = sel[row * k + x];
+                            if (sj < 0 || sj >= dv.C) continue;
+                            const float wx = expf(lse_p[row * S + 1 + x] - M) / Z;
+                            const float4* src = reinterpret_cast<const float4*>(o_p + (row * S + 1 + x) * D + c * 32);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const float4 v = src[i];
+                                acc[4 * i] += wx * v.x;
+                                acc[4 * i + 1] += wx * v.y;
+                                acc[4 * i + 2] += wx * v.z;
+                                acc[4 * i + 3] += wx * v.w;
+                            }
+                        }
+                        uint4* dst4 = reinterpret_cast<uint4*>(O_out + row * D + c * 32);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dst4[i] = make_uint4(pack_bf16(acc[8 * i], acc[8 * i + 1]), pack_bf16(acc[8 * i + 2], acc[8 * i + 3]),
+                                                 pack_bf16(acc[8 * i + 4], acc[8 * i + 5]),
+                                                 pack_bf16(acc[8 * i + 6], acc[8 * i + 7]));
+                    }
+                }
+                tc_fence_before();
+                if (my_tok >= 0 && lse_out) lse_out[row] = M + logf(Z);
+                continue;
+            }
             const float inv = 1.f / l;
             float* dst = (my_tok >= 0) ? o_p + ((size_t(itm.bh) * L + my_tok) * S + my_slot) * D : nullptr;
             float* rdst[8];  // destination row of this lane in store step i: row 4i + lane / 8
@@ -530,6 +537,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_before();
             if (dst) lse_p[(size_t(itm.bh) * L + my_tok) * S + my_slot] = (m_used + log2f(l)) * 0.69314718055994531f;
+            if (FUSED) {
+                // publish this warp's routed rows: every lane's stores, then one count
+                __threadfence();
+                __syncwarp();
+                const unsigned vm = __ballot_sync(0xffffffffu, dst != nullptr);
+                if (lane == 0 && vm) atomicAdd(&hdr[HDR_RDONE], __popc(vm));
+            }
         }
     }
 
@@ -541,14 +555,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int D>
+template <int D, bool FUSED>
 cudaError_t launch_d(const DevLayout& dv, int BH, const void* Q, const void* K, const void* V, int k,
-                     float scale, int64_t n_anchor, char* ws, const WsPlan& p, cudaStream_t s) {
+                     float scale, int64_t n_anchor, char* ws, const WsPlan& p, const int32_t* sel, void* O,
+                     float* lse, cudaStream_t s) {
     CUtensorMap tmK, tmV;
     const int64_t rows = int64_t(BH) * dv.L;
     if (!make_tmap(&tmK, K, D, rows) || !make_tmap(&tmV, V, D, rows)) return cudaErrorInvalidValue;
     const int smem = Cfg<D>::kSmem;
-    cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel<D, FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -556,13 +571,13 @@ cudaError_t launch_d(const DevLayout& dv, int BH, const void* Q, const void* K, 
     const AttendSchedule sched = attend_schedule();
     if (sched.n_ctas > 0 && sched.n_ctas < sms) sms = sched.n_ctas;
     int32_t* hdr = reinterpret_cast<int32_t*>(ws + p.hdr);
-    e = cudaMemsetAsync(hdr + HDR_WORK, 0, sizeof(int32_t), s);
+    e = cudaMemsetAsync(hdr + HDR_WORK, 0, 2 * sizeof(int32_t), s);  // work counter, routed rows done
     if (e != cudaSuccess) return e;
-    attend_tc_kernel<D><<<sms, kThreads, smem, s>>>(
+    attend_tc_kernel<D, FUSED><<<sms, kThreads, smem, s>>>(
         tmK, tmV, dv, BH, k, scale * 1.4426950408889634f, n_anchor, static_cast<const __nv_bfloat16*>(Q), hdr,
         reinterpret_cast<const int32_t*>(ws + p.qoff), reinterpret_cast<const int32_t*>(ws + p.tile_off),
         reinterpret_cast<const int32_t*>(ws + p.qlist), reinterpret_cast<float*>(ws + p.lse_p),
-        reinterpret_cast<float*>(ws + p.o_p), sched.reverse);
+        reinterpret_cast<float*>(ws + p.o_p), sched.reverse, sel, static_cast<__nv_bfloat16*>(O), lse);
     return cudaGetLastError();
 }
 
@@ -571,8 +586,15 @@ cudaError_t launch_d(const DevLayout& dv, int BH, const void* Q, const void* K, 
 cudaError_t launch_attend_tc(const DevLayout& dv, int BH, int d, const void* Q, const void* K,
                              const void* V, int k, float scale, int64_t n_anchor, char* ws,
                              const WsPlan& p, cudaStream_t s) {
-    if (d == 128) return launch_d<128>(dv, BH, Q, K, V, k, scale, n_anchor, ws, p, s);
-    return launch_d<64>(dv, BH, Q, K, V, k, scale, n_anchor, ws, p, s);
+    if (d == 128) return launch_d<128, false>(dv, BH, Q, K, V, k, scale, n_anchor, ws, p, nullptr, nullptr, nullptr, s);
+    return launch_d<64, false>(dv, BH, Q, K, V, k, scale, n_anchor, ws, p, nullptr, nullptr, nullptr, s);
+}
+
+cudaError_t launch_attend_merged(const DevLayout& dv, int BH, int d, const void* Q, const void* K,
+                                 const void* V, int k, float scale, int64_t n_anchor, char* ws,
+                                 const WsPlan& p, const int32_t* sel, void* O, float* lse, cudaStream_t s) {
+    if (d == 128) return launch_d<128, true>(dv, BH, Q, K, V, k, scale, n_anchor, ws, p, sel, O, lse, s);
+    return launch_d<64, true>(dv, BH, Q, K, V, k, scale, n_anchor, ws, p, sel, O, lse, s);
 }
 
 }  // namespace moc

@@ -15,10 +15,11 @@
 // (many candidates) take fewer of them - with NWG selection warpgroups
 // (4 for k <= 8, else 2) and two more warps:
 //   warp 4*NWG (one lane): streams each tile's Q rows (two 64-column,
-//          128-byte-swizzled slabs) into a 2-stage ring with TMA;
+//          128-byte-swizzled slabs) into a ring with TMA (5 stages when every
+//          candidate list fits a 128-row operand block, else 2);
 //   warp 4*NWG+1: owns 512 TMEM columns (one 512/NWG-column score buffer per
-//          selection warpgroup). When the (head, group, 256-candidate operand
-//          block) changes it converts the block's fp32 pooled keys into
+//          selection warpgroup). When the (head, group, 128- or 256-candidate
+//          operand block) changes it converts the block's fp32 pooled keys into
 //          swizzled bf16 operands hi = RN(Kbar) and lo = RN(Kbar - hi) - Q is
 //          exact bf16, so the two bf16 products reproduce q . Kbar to ~2^-17
 //          relative per term - and its lane 0 issues S = Q hi^T + Q lo^T for
@@ -44,7 +45,6 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kBlk = 256;  // candidates per operand block in shared memory
 constexpr int kIdNone = 0x7fffffff;
 
 template <int KMAX>
@@ -55,24 +55,32 @@ struct RWarps {
     static constexpr int kProducer = kNwg * 4, kIssuer = kNwg * 4 + 1;
 };
 
-template <int D>
+// Shared memory of one CTA: a QS-stage ring of 128-row Q tiles and the hi / lo
+// operand blocks of KBLK candidates. Groups with at most 128 candidates (every
+// group of the eight-shot scene has <= 105) use KBLK = 128, which leaves room
+// for a deeper Q ring (more bytes in flight per SM); larger candidate lists use
+// KBLK = 256 and a 2-stage ring.
+template <int D, int KBLK, int QS>
 struct RCfg {
+    static constexpr int kBlk = KBLK;                   // candidates per operand block
     static constexpr int kSlabs = D / 64;
     static constexpr int kQBytes = kSlabs * 128 * 128;  // one 128-row Q tile
-    static constexpr int kKbSlab = kBlk * 128;          // 256 rows x 128 B
+    static constexpr int kKbSlab = KBLK * 128;          // KBLK rows x 128 B
     static constexpr int kKbBytes = kSlabs * kKbSlab;   // hi (or lo) block
-    static constexpr int kQStages = 2;                  // Q ring depth
+    static constexpr int kQStages = QS;                 // Q ring depth
     static constexpr int oQ = 0;
     static constexpr int oHi = oQ + kQStages * kQBytes;
     static constexpr int oLo = oHi + kKbBytes;
     static constexpr int oBar = oLo + kKbBytes;
-    static constexpr int kSmem = (oBar + 256 + 1024) > 120 * 1024 ? (oBar + 256 + 1024) : 120 * 1024;
+    static constexpr int kSmem = (oBar + 512 + 1024) > 120 * 1024 ? (oBar + 512 + 1024) : 120 * 1024;
+    static_assert(QS <= 8, "barrier slots");
+    static_assert(kSmem <= 227 * 1024, "shared memory");
 };
 
 // R_Q_FULL / R_Q_EMPTY: [ring stage]; R_S_FULL / R_S_FREE: [warpgroup]; R_KB_FREE: the MMAs that read the operand block are done
-enum { R_Q_FULL = 0, R_Q_EMPTY = 4, R_S_FULL = 8, R_S_FREE = 12, R_KB_FREE = 16, R_MMA_DONE = 17 };
+enum { R_Q_FULL = 0, R_Q_EMPTY = 8, R_S_FULL = 16, R_S_FREE = 20, R_KB_FREE = 24, R_MMA_DONE = 25 };
 
-struct RShared {  // at oBar + 192 (after the barriers)
+struct RShared {  // at oBar + 256 (after the barriers)
     uint32_t tmem_base;
     int abort;
     int64_t t_beg, t_end;  // this CTA's tile range
@@ -168,7 +176,7 @@ struct TileWalk {
 
 // Fill the hi / lo operand block (K-major, 128-byte swizzle) of candidates
 // [cbeg + b * kBlk, + nbc) of head bh; rows up to npad are zero. Run by one warp.
-template <int D, int KBSLAB>
+template <int D, int KBSLAB, int KBLK>
 __device__ __forceinline__ void build_block(const DevLayout& dv, const float* __restrict__ Kbar, int bh, int cbeg,
                                             int b, int nbc, int npad, uint32_t sHi, uint32_t sLo, int lane) {
     const float* kb = Kbar + size_t(bh) * dv.C * D;
@@ -177,7 +185,7 @@ __device__ __forceinline__ void build_block(const DevLayout& dv, const float* __
         const int r = i / CH, ch = i % CH;
         float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
         if (r < nbc) {
-            const int c = dv.cand[cbeg + b * kBlk + r];
+            const int c = dv.cand[cbeg + b * KBLK + r];
             const float4 a = *reinterpret_cast<const float4*>(kb + size_t(c) * D + ch * 8);
             const float4 bq = *reinterpret_cast<const float4*>(kb + size_t(c) * D + ch * 8 + 4);
             v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
@@ -200,12 +208,13 @@ __device__ __forceinline__ void build_block(const DevLayout& dv, const float* __
     }
 }
 
-template <int D, int KMAX>
+template <int D, int KMAX, int KBLK, int QS>
 __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
     route_tc_kernel(const __grid_constant__ CUtensorMap tmQ, DevLayout dv, int64_t total_tiles,
                     int64_t rtiles, const float* __restrict__ Kbar, int k, int causal,
                     const uint64_t* __restrict__ seg_mask, int32_t* __restrict__ sel) {
-    using C = RCfg<D>;
+    using C = RCfg<D, KBLK, QS>;
+    constexpr int kBlk = C::kBlk;
     using WP = RWarps<KMAX>;
     constexpr int NWG = WP::kNwg, SLICE = WP::kSlice;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -214,7 +223,7 @@ __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
     unsigned char* gbase = smem_raw + (base - raw);
     const uint32_t sQ = base + C::oQ, sHi = base + C::oHi, sLo = base + C::oLo;
     const uint32_t sBar = base + C::oBar;
-    RShared& sh = *reinterpret_cast<RShared*>(gbase + C::oBar + 192);
+    RShared& sh = *reinterpret_cast<RShared*>(gbase + C::oBar + 256);
     volatile int* abort = &sh.abort;
     int32_t* err = dv.err;
     auto bar = [&](int i) { return sBar + 8u * uint32_t(i); };
@@ -304,8 +313,8 @@ __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
                         ++nkb;
                     }
                     const int nbk = min(kBlk, x.ncand - kb * kBlk);
-                    build_block<D, C::kKbSlab>(dv, Kbar, x.bh, x.cbeg, kb, nbk, (nbk + 15) & ~15, sHi, sLo,
-                                               lane);
+                    build_block<D, C::kKbSlab, kBlk>(dv, Kbar, x.bh, x.cbeg, kb, nbk, (nbk + 15) & ~15, sHi,
+                                                     sLo, lane);
                     fence_proxy_async_smem();
                     __syncwarp();
                     last_bh = x.bh; last_g = x.g; last_b = kb;
@@ -415,48 +424,63 @@ __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
     }
 }
 
-template <int D, int KMAX>
-cudaError_t launch_dk(const DevLayout& dv, int BH, int64_t rtiles, const void* Q, const float* Kbar, int k,
-                      int causal, const uint64_t* seg_mask, int32_t* sel, cudaStream_t s) {
+template <int D, int KMAX, int KBLK, int QS>
+cudaError_t launch_cfg(const DevLayout& dv, int BH, int64_t rtiles, const void* Q, const float* Kbar, int k,
+                       int causal, const uint64_t* seg_mask, int32_t* sel, cudaStream_t s) {
     CUtensorMap tmQ;
     if (!make_tmap(&tmQ, Q, D, int64_t(BH) * dv.L)) return cudaErrorInvalidValue;
-    const int smem = RCfg<D>::kSmem;
-    cudaError_t e = cudaFuncSetAttribute(route_tc_kernel<D, KMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const int smem = RCfg<D, KBLK, QS>::kSmem;
+    cudaError_t e = cudaFuncSetAttribute(route_tc_kernel<D, KMAX, KBLK, QS>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t total = int64_t(BH) * rtiles;
     const int grid = int(total < sms ? total : sms);
-    route_tc_kernel<D, KMAX><<<grid, RWarps<KMAX>::kThreads, smem, s>>>(tmQ, dv, total, rtiles, Kbar, k, causal,
-                                                                        seg_mask, sel);
+    route_tc_kernel<D, KMAX, KBLK, QS><<<grid, RWarps<KMAX>::kThreads, smem, s>>>(tmQ, dv, total, rtiles, Kbar, k,
+                                                                                  causal, seg_mask, sel);
     return cudaGetLastError();
+}
+
+// Candidate lists of at most 128 entries fit one 128-row operand block, which
+// frees shared memory for a 5-stage Q ring; longer lists take 256-row blocks and
+// a 2-stage ring. (With 2 selection warpgroups a slice is 256 candidates, which
+// needs the 256-row block.)
+template <int D, int KMAX>
+cudaError_t launch_dk(const DevLayout& dv, int BH, int64_t rtiles, const void* Q, const float* Kbar, int k,
+                      int causal, int max_cand, const uint64_t* seg_mask, int32_t* sel, cudaStream_t s) {
+    if constexpr (RWarps<KMAX>::kSlice <= 128) {
+        if (max_cand <= 128)
+            return launch_cfg<D, KMAX, 128, 5>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
+    }
+    return launch_cfg<D, KMAX, 256, 2>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
 }
 
 template <int D>
 cudaError_t launch_d(const DevLayout& dv, int BH, int64_t rtiles, const void* Q, const float* Kbar, int k,
-                     int causal, const uint64_t* seg_mask, int32_t* sel, cudaStream_t s) {
+                     int causal, int max_cand, const uint64_t* seg_mask, int32_t* sel, cudaStream_t s) {
     // exact list length for small k (the insertion network costs one level per entry)
     switch (k) {
-        case 1: return launch_dk<D, 1>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
-        case 2: return launch_dk<D, 2>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
-        case 3: return launch_dk<D, 3>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
-        case 4: return launch_dk<D, 4>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
+        case 1: return launch_dk<D, 1>(dv, BH, rtiles, Q, Kbar, k, causal, max_cand, seg_mask, sel, s);
+        case 2: return launch_dk<D, 2>(dv, BH, rtiles, Q, Kbar, k, causal, max_cand, seg_mask, sel, s);
+        case 3: return launch_dk<D, 3>(dv, BH, rtiles, Q, Kbar, k, causal, max_cand, seg_mask, sel, s);
+        case 4: return launch_dk<D, 4>(dv, BH, rtiles, Q, Kbar, k, causal, max_cand, seg_mask, sel, s);
         default: break;
     }
-    if (k <= 8) return launch_dk<D, 8>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
-    if (k <= 16) return launch_dk<D, 16>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
-    return launch_dk<D, 32>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
+    if (k <= 8) return launch_dk<D, 8>(dv, BH, rtiles, Q, Kbar, k, causal, max_cand, seg_mask, sel, s);
+    if (k <= 16) return launch_dk<D, 16>(dv, BH, rtiles, Q, Kbar, k, causal, max_cand, seg_mask, sel, s);
+    return launch_dk<D, 32>(dv, BH, rtiles, Q, Kbar, k, causal, max_cand, seg_mask, sel, s);
 }
 
 }  // namespace
 
 cudaError_t launch_route(const DevLayout& dv, int BH, int64_t rtiles, int d, const void* Q,
-                         const float* Kbar, int k, int causal, const uint64_t* seg_mask, int32_t* sel,
-                         cudaStream_t s) {
+                         const float* Kbar, int k, int causal, int max_cand, const uint64_t* seg_mask,
+                         int32_t* sel, cudaStream_t s) {
     if (rtiles <= 0 || BH > 65535) return cudaErrorInvalidValue;
-    if (d == 128) return launch_d<128>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
-    return launch_d<64>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
+    if (d == 128) return launch_d<128>(dv, BH, rtiles, Q, Kbar, k, causal, max_cand, seg_mask, sel, s);
+    return launch_d<64>(dv, BH, rtiles, Q, Kbar, k, causal, max_cand, seg_mask, sel, s);
 }
 
 }  // namespace moc

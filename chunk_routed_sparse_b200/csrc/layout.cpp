@@ -203,6 +203,53 @@ moc_status build_host(const moc_layout_desc* d, moc_layout* lay) {
         lay->atile_off.push_back(lay->atile_off.back() + (nq + moc::kItemRows - 1) / moc::kItemRows);
     }
     lay->total_atiles = lay->atile_off.back();
+
+    // Key blocks of the backward pass. Every key is attended by the queries of the
+    // groups whose anchor ranges hold it and, for a video chunk, by the queries that
+    // selected that chunk. A video chunk is its own block (its selecting queries
+    // are its own); consecutive caption chunks attended by the same groups (every
+    // group: captions are mandatory for all queries) form one block.
+    std::vector<std::vector<int32_t>> anch(n);
+    for (int g = 0; g < G; ++g) {
+        for (int r = lay->ar_off[g]; r < lay->ar_off[g + 1]; ++r) {
+            const int32_t a = lay->ar[2 * r], b = lay->ar[2 * r + 1];
+            int c = int(std::upper_bound(lay->chunk_off.begin(), lay->chunk_off.end(), a) - lay->chunk_off.begin()) - 1;
+            for (; c < n && lay->chunk_off[c] < b; ++c) anch[c].push_back(g);
+        }
+    }
+    lay->kb_range.clear();
+    lay->kb_chunk.clear();
+    lay->kb_goff.assign(1, 0);
+    lay->kb_grp.clear();
+    std::vector<int64_t> kb_rows;  // anchoring query rows of every block
+    for (int c = 0; c < n;) {
+        int e = c + 1;
+        if (lay->kind[c] == MOC_CAPTION)
+            while (e < n && lay->kind[e] == MOC_CAPTION && anch[e] == anch[c]) ++e;
+        lay->kb_range.push_back(lay->chunk_off[c]);
+        lay->kb_range.push_back(lay->chunk_off[e]);
+        lay->kb_chunk.push_back(lay->kind[c] == MOC_VIDEO ? c : -1);
+        int64_t rows = 0;
+        for (int32_t g : anch[c]) {
+            lay->kb_grp.push_back(g);
+            rows += lay->grp_q1[g] - lay->grp_q0[g];
+        }
+        lay->kb_goff.push_back(int32_t(lay->kb_grp.size()));
+        kb_rows.push_back(rows);
+        c = e;
+    }
+    const int NKB = int(kb_rows.size());
+    lay->kb_order.resize(NKB);
+    std::iota(lay->kb_order.begin(), lay->kb_order.end(), 0);
+    std::stable_sort(lay->kb_order.begin(), lay->kb_order.end(),
+                     [&](int x, int y) { return kb_rows[x] > kb_rows[y]; });
+    lay->kt_off.assign(1, 0);
+    for (int x = 0; x < NKB; ++x) {
+        const int b = lay->kb_order[x];
+        const int32_t nk = lay->kb_range[2 * b + 1] - lay->kb_range[2 * b];
+        lay->kt_off.push_back(lay->kt_off.back() + (nk + moc::kQTile - 1) / moc::kQTile);
+    }
+    lay->total_ktiles = lay->kt_off.back();
     return MOC_OK;
 }
 
@@ -211,7 +258,8 @@ moc_status upload(moc_layout* lay) {
         &lay->chunk_off, &lay->grp_q0, &lay->grp_q1, &lay->grp_kind, &lay->ar_off, &lay->ar,
         &lay->cand_off, &lay->cand, &lay->cand_ncausal, &lay->rtile_off, &lay->atile_off,
         &lay->a_order, &lay->cand_seg, &lay->grp_seg, &lay->seg_voff, &lay->vid,
-        &lay->rcost_full, &lay->rcost_causal};
+        &lay->rcost_full, &lay->rcost_causal, &lay->kb_range, &lay->kb_chunk, &lay->kb_goff,
+        &lay->kb_grp, &lay->kb_order, &lay->kt_off};
     std::vector<size_t> offs;
     size_t total = 0;
     for (auto* t : tabs) {
@@ -257,6 +305,13 @@ moc_status upload(moc_layout* lay) {
     dv.vid = at(15);
     dv.rcost[0] = at(16);
     dv.rcost[1] = at(17);
+    dv.NKB = int32_t(lay->kb_chunk.size());
+    dv.kb_range = at(18);
+    dv.kb_chunk = at(19);
+    dv.kb_goff = at(20);
+    dv.kb_grp = at(21);
+    dv.kb_order = at(22);
+    dv.kt_off = at(23);
     dv.err = reinterpret_cast<int32_t*>(static_cast<char*>(lay->dev_block) + err_off);
     return MOC_OK;
 }
@@ -345,6 +400,12 @@ extern "C" moc_status moc_layout_table(const moc_layout* layout, int which, int3
         case 10: src = &layout->vid; break;
         case 11: src = &layout->rcost_full; break;
         case 12: src = &layout->rcost_causal; break;
+        case 13: src = &layout->kb_range; break;
+        case 14: src = &layout->kb_chunk; break;
+        case 15: src = &layout->kb_goff; break;
+        case 16: src = &layout->kb_grp; break;
+        case 17: src = &layout->kb_order; break;
+        case 18: src = &layout->kt_off; break;
         default: return MOC_ERR_INVALID_ARG;
     }
     *count = int64_t(src->size());

@@ -38,6 +38,15 @@ struct DevLayout {
     const int32_t* vid;          // video chunk ids in stream order
     const int32_t* rcost[2];     // [rtiles+1] prefix of estimated router tile costs, full / causal lists
     int32_t* err;                // [2] error word + detail of kernels without a workspace (router)
+    // backward (key-major dK / dV): key blocks = a video chunk, or a run of caption
+    // chunks that the same query groups attend
+    int32_t NKB;
+    const int32_t* kb_range;     // [NKB][2] token range (k0, k1) of every key block
+    const int32_t* kb_chunk;     // [NKB] video chunk whose query list also attends it (-1: caption run)
+    const int32_t* kb_goff;      // [NKB+1] offsets into kb_grp
+    const int32_t* kb_grp;       // query groups whose anchor ranges hold the block
+    const int32_t* kb_order;     // [NKB] blocks by descending anchoring query rows
+    const int32_t* kt_off;       // [NKB+1] prefix of 128-key tiles over kb_order
 };
 
 }  // namespace moc
@@ -55,6 +64,8 @@ struct moc_layout {
     std::vector<int32_t> cand_seg, grp_seg, seg_voff, vid;  // segments (shots) in stream order
     std::vector<int32_t> rcost_full, rcost_causal;          // router tile cost prefixes
     std::vector<int64_t> grp_keys;  // anchor keys of each group
+    std::vector<int32_t> kb_range, kb_chunk, kb_goff, kb_grp, kb_order, kt_off;  // backward key blocks
+    int64_t total_ktiles = 0;       // 128-key tiles per (b, h)
     void* dev_block = nullptr;
     moc::DevLayout dv{};
 };
@@ -75,7 +86,7 @@ struct WsPlan {
 };
 WsPlan plan_workspace(const moc_layout* lay, int B, int H, int d, int k);
 
-enum { HDR_ERR = 0, HDR_DETAIL = 1, HDR_WORK = 2 };
+enum { HDR_ERR = 0, HDR_DETAIL = 1, HDR_WORK = 2, HDR_RDONE = 3 };
 enum { ERR_NONE = 0, ERR_TIMEOUT = 1, ERR_CHECK = 2 };
 
 // Work schedule of the attention kernel (moc_set_attend_schedule): CTAs
@@ -91,8 +102,8 @@ AttendSchedule attend_schedule();
 cudaError_t launch_pool(const DevLayout& dv, int BH, int d, const void* K, float* Kbar,
                         cudaStream_t s);
 cudaError_t launch_route(const DevLayout& dv, int BH, int64_t rtiles, int d, const void* Q,
-                         const float* Kbar, int k, int causal, const uint64_t* seg_mask, int32_t* sel,
-                         cudaStream_t s);
+                         const float* Kbar, int k, int causal, int max_cand, const uint64_t* seg_mask,
+                         int32_t* sel, cudaStream_t s);
 cudaError_t launch_outer(const DevLayout& dv, int BH, int d, const float* Qbar, const float* Kbar, int M,
                          int causal, uint64_t* seg_mask, cudaStream_t s);
 cudaError_t launch_qlists(const DevLayout& dv, int BH, int k, const int32_t* sel, char* ws,
@@ -100,8 +111,26 @@ cudaError_t launch_qlists(const DevLayout& dv, int BH, int k, const int32_t* sel
 cudaError_t launch_attend_tc(const DevLayout& dv, int BH, int d, const void* Q, const void* K,
                              const void* V, int k, float scale, int64_t n_anchor_items, char* ws,
                              const WsPlan& p, cudaStream_t s);
+cudaError_t launch_attend_merged(const DevLayout& dv, int BH, int d, const void* Q, const void* K,
+                                 const void* V, int k, float scale, int64_t n_anchor, char* ws,
+                                 const WsPlan& p, const int32_t* sel, void* O, float* lse, cudaStream_t s);
 cudaError_t launch_merge(int BH, int L, int d, int k, const int32_t* sel, void* O, float* lse,
                          const char* ws, const WsPlan& p, cudaStream_t s);
+
+// Backward pass (dQ, dK, dV). The workspace holds the forward plan's header and
+// query lists; lse_p holds D = dO . o per row (fp32 [BH][L]) and o_p the dQ
+// partial rows (fp32 [BH][L][1+k][d]).
+WsPlan plan_workspace_bwd(const moc_layout* lay, int B, int H, int d, int k);
+cudaError_t launch_bwd_rowdot(int BH, int L, int d, const void* O, const void* dO, char* ws, const WsPlan& p,
+                              cudaStream_t s);
+cudaError_t launch_bwd_dq(const DevLayout& dv, int BH, int d, const void* Q, const void* K, const void* V,
+                          const void* dO, const float* lse, int k, float scale, int64_t n_anchor, char* ws,
+                          const WsPlan& p, cudaStream_t s);
+cudaError_t launch_bwd_dq_reduce(int BH, int L, int C, int d, int k, const int32_t* sel, void* dQ, const char* ws,
+                                 const WsPlan& p, cudaStream_t s);
+cudaError_t launch_bwd_dkv(const DevLayout& dv, int BH, int d, const void* Q, const void* K, const void* V,
+                           const void* dO, const float* lse, float scale, char* ws, const WsPlan& p, void* dK,
+                           void* dV, cudaStream_t s);
 
 // Poisson distribution function at 0 .. m_max-1 scaled to 2^32 (drop-in counts)
 struct PoissonThresholds {

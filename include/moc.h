@@ -114,7 +114,13 @@ moc_status moc_layout_info(const moc_layout* layout, int64_t* L, int32_t* C, int
  *        group's queries [G] (-1: caption group), 9 offsets of every segment's
  *        video chunks in table 10 [S+1], 10 video chunk ids in stream order,
  *        11 / 12 prefix of the router's estimated tile costs for the full /
- *        causal candidate lists [router tiles + 1].
+ *        causal candidate lists [router tiles + 1],
+ *        backward key blocks (a video chunk, or a run of caption chunks the
+ *        same groups attend): 13 token range (k0,k1)[NKB][2], 14 video chunk
+ *        of the block or -1 [NKB], 15 offsets into table 16 [NKB+1], 16 query
+ *        groups whose anchor ranges hold the block, 17 blocks by descending
+ *        anchoring query rows [NKB], 18 prefix of 128-key tiles over table 17
+ *        [NKB+1].
  * Writes min(count, cap) int32 values to out (may be NULL with cap 0) and
  * the full count to *count. */
 moc_status moc_layout_table(const moc_layout* layout, int which, int32_t* out, int64_t cap,
@@ -217,6 +223,18 @@ moc_status moc_attend_partials(const moc_layout* layout, int B, int H, int d, co
                                const void* K, const void* V, int k, float softmax_scale,
                                void* ws, size_t ws_bytes, moc_stream_t stream);
 
+/* (4) and (5) in one kernel: the attention of (4) with the merge of (5) done in
+ * place. Routed items run first and write their partials; each anchor item
+ * then combines its own part (kept in TMEM, never written) with its rows'
+ * routed partials by the log-sum-exp rule of (5), in the same fixed slot order,
+ * and writes the bf16 output row and lse (nullable) itself - the anchor
+ * partials are never stored or read back. An entry of sel outside [0, C) is
+ * skipped. Needs the workspace filled by (3) for the same sel. */
+moc_status moc_attend_merged(const moc_layout* layout, int B, int H, int d, const void* Q,
+                             const void* K, const void* V, const int32_t* sel, int k,
+                             float softmax_scale, void* O, float* lse, void* ws, size_t ws_bytes,
+                             moc_stream_t stream);
+
 /* (5) Log-sum-exp merge of every query's partials (Summary §3.1: softmax
  * attention over Omega(q); Omega(q) is a disjoint union of the anchor keys and
  * the selected chunks, and softmax over a disjoint union equals the
@@ -229,8 +247,8 @@ moc_status moc_merge(const moc_layout* layout, int B, int H, int d, int k, const
                      void* O, float* lse, void* ws, size_t ws_bytes, moc_stream_t stream);
 
 /* Full attention stage (Summary §3.1: o = Softmax(q K_Omega^T / sqrt(d))
- * V_Omega over Omega(q) = anchors + the chunks in sel): (3), (4) and (5) in
- * order on one stream. sel: device int32 [B][H][L][k] from (2) or (2'),
+ * V_Omega over Omega(q) = anchors + the chunks in sel): (3), then (4) and (5)
+ * fused (moc_attend_merged), on one stream. sel: device int32 [B][H][L][k] from (2) or (2'),
  * -1 padded (NULL when k == 0); O: device bf16 [B][H][L][d]; lse: device fp32
  * [B][H][L] (nullable); ws: the caller's workspace, 256-byte aligned, of at
  * least moc_attention_workspace_bytes() bytes. */
@@ -238,6 +256,35 @@ moc_status moc_attention_fwd(const moc_layout* layout, int B, int H, int d, cons
                              const void* K, const void* V, const int32_t* sel, int k,
                              float softmax_scale, void* O, float* lse, void* ws,
                              size_t ws_bytes, moc_stream_t stream);
+
+/* Bytes of device workspace moc_attention_bwd needs (0 on invalid arguments):
+ * the query lists of (3), D = dO . o per row and the dQ partial rows (1+k fp32
+ * rows of d per query). */
+size_t moc_attention_bwd_workspace_bytes(const moc_layout* layout, int B, int H, int d, int k);
+
+/* Backward pass of the attention stage: dQ, dK, dV for an upstream gradient dO
+ * of O ("Mixture of Contexts for Long Video Generation | Summary", appendix on
+ * training: the model is trained through a custom autograd function of the
+ * attention over the selected keys and values; the top-k choice is discrete
+ * and is not differentiated). The selection sel is a constant, so no gradient
+ * reaches the pooled keys, and the loss depends on O only (no gradient on lse).
+ * With p_tu = exp(scale q_t.k_u - lse_t) over u in Omega(t) and
+ * D_t = dO_t . O_t:
+ *   ds_tu = p_tu (dO_t . v_u - D_t),   dQ_t = scale sum_u ds_tu k_u,
+ *   dK_u = scale sum_t ds_tu q_t,      dV_u = sum_t p_tu dO_t.
+ * Q, K, V, O, dO: device bf16 [B][H][L][d] (O from the forward pass); lse:
+ * device fp32 [B][H][L], the forward pass's log-sum-exp; sel: as for
+ * moc_attention_fwd (the selection the forward pass used); dQ, dK, dV: device
+ * bf16 [B][H][L][d] outputs, accumulated in fp32 and rounded to nearest even.
+ * ws: 256-byte aligned, at least moc_attention_bwd_workspace_bytes() bytes.
+ * Deterministic: dQ is summed per row from per-part partials in fixed order;
+ * each key's dK and dV are accumulated by one CTA over a fixed query order.
+ * Asynchronous on the stream; device errors as for moc_attention_fwd. */
+moc_status moc_attention_bwd(const moc_layout* layout, int B, int H, int d, const void* Q,
+                             const void* K, const void* V, const void* O, const float* lse,
+                             const void* dO, const int32_t* sel, int k, float softmax_scale,
+                             void* dQ, void* dK, void* dV, void* ws, size_t ws_bytes,
+                             moc_stream_t stream);
 
 /* moc_attention_fwd without a caller workspace, for callers that cannot
  * allocate device memory (a plugin given only its input and output buffers, a

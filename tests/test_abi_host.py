@@ -199,3 +199,44 @@ def test_segment_tables_agree_with_oracle(wl):
         assert pre[0] == 0 and all(b > a for a, b in zip(pre, pre[1:]))
         ntiles = sum((grp[2 * g + 1] - grp[2 * g] + 127) // 128 for g in range(len(grp) // 2))
         assert len(pre) == ntiles + 1
+
+
+@pytest.mark.parametrize("wl", WORKLOADS + RANDOM[:80], ids=lambda w: f"{w.name}-{w.anchor}")
+def test_backward_key_blocks_agree_with_oracle_roles(wl):
+    """Key blocks of the backward pass: they tile the token stream in order;
+    each is one video chunk or a run of caption chunks; its group list is
+    exactly the groups whose queries hold every chunk of the block as an
+    anchor (oracle role table); blocks are ordered by descending anchoring
+    query rows and the tile prefix counts 128-key tiles in that order."""
+    lay = _host_layout(wl)
+    orc = oracle.Layout(wl)
+    rng_ = np.array(lay.table(13)).reshape(-1, 2)
+    kb_chunk, kb_goff, kb_grp = lay.table(14), lay.table(15), lay.table(16)
+    kb_order, kt_off = lay.table(17), lay.table(18)
+    grp = np.array(lay.table(1)).reshape(-1, 2)
+    nkb = len(kb_chunk)
+    assert rng_[0, 0] == 0 and rng_[-1, 1] == orc.L and np.all(rng_[1:, 0] == rng_[:-1, 1])
+    rows = []
+    for b in range(nkb):
+        k0, k1 = rng_[b]
+        chunks = sorted(set(orc.chunk_of_token[k0:k1].tolist()))
+        assert orc.off[chunks[0]] == k0 and orc.off[chunks[-1] + 1] == k1
+        if kb_chunk[b] >= 0:
+            assert chunks == [kb_chunk[b]] and orc.kind[kb_chunk[b]] == W.VIDEO
+        else:
+            assert all(orc.kind[c] == W.CAPTION for c in chunks)
+        want = set()
+        for g, (q0, q1) in enumerate(grp):
+            qc = int(orc.chunk_of_token[q0])
+            hold = [orc.role[qc, c] == oracle.ROLE_ANCHOR for c in chunks]
+            assert all(hold) or not any(hold), (b, g)
+            if all(hold):
+                want.add(g)
+        got = kb_grp[kb_goff[b]:kb_goff[b + 1]]
+        assert len(set(got)) == len(got) and set(got) == want, (b, got, want)
+        rows.append(sum(grp[g, 1] - grp[g, 0] for g in got))
+    assert sorted(kb_order) == list(range(nkb))
+    assert all(rows[a] >= rows[b] for a, b in zip(kb_order, kb_order[1:]))
+    assert kt_off[0] == 0 and len(kt_off) == nkb + 1
+    for x, b in enumerate(kb_order):
+        assert kt_off[x + 1] - kt_off[x] == (rng_[b, 1] - rng_[b, 0] + 127) // 128

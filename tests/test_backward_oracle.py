@@ -64,3 +64,24 @@ def test_value_gradient_sums_to_upstream():
     sel = oracle.route(wl, Q, oracle.pool(wl, K, lay), lay=lay)["sel"]
     _, _, dV = BW.backward(wl, lay, Q, K, V, sel, dO)
     np.testing.assert_allclose(dV.sum(axis=2), dO.numpy().sum(axis=2), rtol=0, atol=1e-9)
+
+
+@pytest.mark.parametrize("anchor,causal,k", [("shot", True, 2), ("local", True, 1), ("chunk", False, 3)])
+def test_row_and_key_samples_match_the_full_backward(anchor, causal, k):
+    """backward_rows and backward_keys (the sampled forms used on large scenes)
+    equal the full backward on the rows / keys they cover, for every chunk
+    kind: caption chunks (attended by every query), and video chunks attended
+    as anchors and as selections."""
+    wl = W.tiny().replace(anchor=anchor, radius=1, causal=causal, H=2).with_k(k)
+    Q, K, V, dO = _grad_case(wl, 6)
+    lay = oracle.Layout(wl)
+    sel = oracle.route(wl, Q, oracle.pool(wl, K, lay), lay=lay)["sel"]
+    dQ, dK, dV = BW.backward(wl, lay, Q, K, V, sel, dO)
+    rows = np.array([0, 63, 64, 300, 1111, wl.L - 1])
+    np.testing.assert_allclose(BW.backward_rows(wl, lay, Q, K, V, sel, dO, rows), dQ[:, :, rows],
+                               rtol=0, atol=1e-10)
+    for b, h, c in [(0, 0, 0), (0, 1, 2), (0, 0, 5), (0, 1, lay.C - 1)]:
+        dk, dv = BW.backward_keys(wl, lay, Q, K, V, sel, dO, b, h, c)
+        u = slice(lay.off[c], lay.off[c + 1])
+        np.testing.assert_allclose(dk, dK[b, h, u], rtol=0, atol=1e-10)
+        np.testing.assert_allclose(dv, dV[b, h, u], rtol=0, atol=1e-10)
