@@ -1,10 +1,9 @@
 """Benchmark of the MoC sparse-attention forward pass (one JSON line on rank 0).
 
 A step is one pass of the whole hot path over one scene: (1) pool keys,
-(2) route, (3) build query lists, (4) attend with (5) the log-sum-exp merge
-fused into it (moc_attend_merged, the path moc_attention_fwd takes). The
-unfused stage calls - (4) writing every partial, then (5) as its own kernel -
-are timed once after the steps for the per-kernel roofline of (5). Default workload:
+(2) route, (3) build query lists, (4) attend, (5) merge - the stage calls
+moc_attention_fwd makes. The variant with (5) fused into (4)
+(moc_attend_merged) is timed once after the steps, beside it. Default workload:
 the eight-shot 180,512-token scene (B=1, H=24, d=128, k=3). Inputs are larger
 than L2 (3 x 1.1 GB), so no L2 flush is needed between steps.
 
@@ -41,8 +40,8 @@ sys.path.insert(0, ROOT)
 import moc_workloads as W  # noqa: E402
 
 METRIC = "MoC fwd tokens/s and selected-pair TFLOP/s (% bf16 peak) at 180k tokens"
-STAGES = ["pool", "route", "qlist", "attend"]  # attend = (4) with the merge (5) fused in
-LAUNCHES_PER_STEP = {"pool": 1, "route": 1, "qlist": 4, "attend": 1}
+STAGES = ["pool", "route", "qlist", "attend", "merge"]
+LAUNCHES_PER_STEP = {"pool": 1, "route": 1, "qlist": 4, "attend": 1, "merge": 1}
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -262,8 +261,10 @@ def run_ours(args):
         if ev: ev[2].record(stream)
         moc.build_qlists(lay, sel, B, H, k, ws)
         if ev: ev[3].record(stream)
-        moc.attend_merged(lay, Q, K, V, sel, k, ws, O, lse, scale)
+        moc.attend_partials(lay, Q, K, V, k, ws, scale)
         if ev: ev[4].record(stream)
+        moc.merge(lay, sel, k, ws, O, lse)
+        if ev: ev[5].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -294,7 +295,7 @@ def run_ours(args):
     stage_ms = {s: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
                 for j, s in enumerate(STAGES)}
     moc.check_device_error(ws)
-    unfused = unfused_timing(moc, lay, Q, K, V, sel, k, ws, scale, stream, B, H, L, d)
+    fused = fused_timing(moc, lay, Q, K, V, sel, k, ws, scale, stream, B, H, L)
 
     # end to end through the C ABI's host-buffer call (moc_forward_host): pinned host
     # Q, K, V in, host O back; inside, chunks of heads are uploaded, computed and
@@ -377,9 +378,9 @@ def run_ours(args):
                      "peak_kind": f"bf16_tflops_sustained ({peak_src})",
                      "frac_of_burst": achieved_tf / float(peaks.get("bf16_tflops", 1590.0)),
                      "traffic": traffic},
-        "hbm_kernels": hbm_fracs(dict(stage_ms, merge=unfused["merge_ms"]), B, H, L, lay.C, d, k, peaks,
-                                 routed_rows(lay, wl), int((sel >= 0).sum().item()) if k > 0 else 0),
-        "unfused_stage_calls": unfused,
+        "hbm_kernels": hbm_fracs(stage_ms, B, H, L, lay.C, d, k, peaks, routed_rows(lay, wl),
+                                 int((sel >= 0).sum().item()) if k > 0 else 0),
+        "fused_attend_merge": fused,
         "clocks": clk,
         "e2e": {"value": job_tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                 "ms_per_step": e2e_ms,
@@ -453,35 +454,32 @@ def dense_compare(moc, wl, Q, K, V, O, lse, stream, moc_pairs, stage_ms, moc_ste
                      "tflops": 4.0 * d * pairs / (a / 1e3) / 1e12,
                      "frac_sustained": 4.0 * d * pairs / (a / 1e3) / 1e12 / peak_tf}
         del ws
-    moc_attention_ms = stage_ms["qlist"] + stage_ms["attend"]
+    moc_attention_ms = stage_ms["qlist"] + stage_ms["attend"] + stage_ms["merge"]
     out["moc_pairs"] = moc_pairs
     out["moc_step_speedup_vs_dense"] = out["dense"]["step_ms"] / moc_step_ms
     out["moc_attention_vs_flop_matched"] = moc_attention_ms / out["flop_matched"]["attention_ms"]
     return out
 
 
-def unfused_timing(moc, lay, Q, K, V, sel, k, ws, scale, stream, B, H, L, d, reps=3):
-    """The stage calls of the unfused path after the timed steps: (4) writing
-    every partial (moc_attend_partials), then (5) as its own kernel (moc_merge);
-    mean of ``reps`` after one untimed run."""
+def fused_timing(moc, lay, Q, K, V, sel, k, ws, scale, stream, B, H, L, reps=3):
+    """(4) with the merge (5) fused into its anchor items' epilogue
+    (moc_attend_merged) after the timed steps, on the same query lists; mean of
+    ``reps`` after one untimed run, against the step's (4) + (5)."""
     O2 = torch.empty_like(Q)
     lse2 = torch.empty(B, H, L, dtype=torch.float32, device=Q.device)
-    att, mer = [], []
+    ts = []
+    moc.build_qlists(lay, sel, B, H, k, ws)
     for it in range(1 + reps):
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-        moc.build_qlists(lay, sel, B, H, k, ws)
-        ev[0].record(stream)
-        moc.attend_partials(lay, Q, K, V, k, ws, scale)
-        ev[1].record(stream)
-        moc.merge(lay, sel, k, ws, O2, lse2)
-        ev[2].record(stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        moc.attend_merged(lay, Q, K, V, sel, k, ws, O2, lse2, scale)
+        e1.record(stream)
         torch.cuda.synchronize()
         if it >= 1:
-            att.append(ev[0].elapsed_time(ev[1]))
-            mer.append(ev[1].elapsed_time(ev[2]))
+            ts.append(e0.elapsed_time(e1))
     moc.check_device_error(ws)
     del O2, lse2
-    return {"attend_partials_ms": statistics.mean(att), "merge_ms": statistics.mean(mer)}
+    return {"attend_merged_ms": statistics.mean(ts)}
 
 
 def backward_timing(moc, lay, Q, K, V, O, lse, sel, k, pairs, d, stream, reps=5):

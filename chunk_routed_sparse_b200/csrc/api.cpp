@@ -271,7 +271,9 @@ extern "C" moc_status moc_attention_fwd(const moc_layout* lay, int B, int H, int
     if (lse && (reinterpret_cast<uintptr_t>(lse) & 3)) return MOC_ERR_INVALID_ARG;
     if (!(scale > 0.0f) || scale != scale) return MOC_ERR_INVALID_ARG;
     if ((st = moc_build_qlists(lay, B, H, k, sel, ws, ws_bytes, stream)) != MOC_OK) return st;
-    return moc_attend_merged(lay, B, H, d, Q, K, V, sel, k, scale, O, lse, ws, ws_bytes, stream);
+    if ((st = moc_attend_partials(lay, B, H, d, Q, K, V, k, scale, ws, ws_bytes, stream)) != MOC_OK)
+        return st;
+    return moc_merge(lay, B, H, d, k, sel, O, lse, ws, ws_bytes, stream);
 }
 
 extern "C" moc_status moc_check_device_error(void* ws, size_t ws_bytes, int32_t* detail,

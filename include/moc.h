@@ -229,7 +229,10 @@ moc_status moc_attend_partials(const moc_layout* layout, int B, int H, int d, co
  * routed partials by the log-sum-exp rule of (5), in the same fixed slot order,
  * and writes the bf16 output row and lse (nullable) itself - the anchor
  * partials are never stored or read back. An entry of sel outside [0, C) is
- * skipped. Needs the workspace filled by (3) for the same sel. */
+ * skipped. Needs the workspace filled by (3) for the same sel. It moves ~4 GB
+ * less through HBM on the eight-shot scene than (4) + (5), but the partial
+ * reads sit in the softmax warps' epilogue, and on one B200 it measured no
+ * faster than (4) + (5); moc_attention_fwd uses (4) + (5). */
 moc_status moc_attend_merged(const moc_layout* layout, int B, int H, int d, const void* Q,
                              const void* K, const void* V, const int32_t* sel, int k,
                              float softmax_scale, void* O, float* lse, void* ws, size_t ws_bytes,
@@ -247,8 +250,8 @@ moc_status moc_merge(const moc_layout* layout, int B, int H, int d, int k, const
                      void* O, float* lse, void* ws, size_t ws_bytes, moc_stream_t stream);
 
 /* Full attention stage (Summary §3.1: o = Softmax(q K_Omega^T / sqrt(d))
- * V_Omega over Omega(q) = anchors + the chunks in sel): (3), then (4) and (5)
- * fused (moc_attend_merged), on one stream. sel: device int32 [B][H][L][k] from (2) or (2'),
+ * V_Omega over Omega(q) = anchors + the chunks in sel): (3), (4) and (5) in
+ * order on one stream (measured faster than (3) + moc_attend_merged). sel: device int32 [B][H][L][k] from (2) or (2'),
  * -1 padded (NULL when k == 0); O: device bf16 [B][H][L][d]; lse: device fp32
  * [B][H][L] (nullable); ws: the caller's workspace, 256-byte aligned, of at
  * least moc_attention_workspace_bytes() bytes. */

@@ -347,3 +347,39 @@ def test_selection_entry_that_is_not_a_chunk_is_reported():
     assert ei.value.status == 7
     moc.attention_fwd(lay, Q, K, V, sel, 2, ws=ws)
     assert moc.check_device_error(ws) == 0
+
+
+@pytest.mark.parametrize("which", ["tiny", "ragsmall"])
+def test_fused_attend_merge_matches_oracle(which):
+    """moc_attend_merged ((4) with (5) in the anchor items' epilogue) against
+    the oracle on every row, under the default and a reversed schedule."""
+    if which == "tiny":
+        wl = W.tiny()
+    else:
+        segs = [W.Segment(37, W.CAPTION, 0, -1)]
+        for i, ln in enumerate([1, 64, 65, 127, 128, 129, 200, 3, 300, 17]):
+            segs.append(W.Segment(ln, W.VIDEO, i // 4, i % 4))
+        wl = W.custom("ragsmall", 2, 3, 128, segs, "shot", 0, True, 3, 31, "frame")
+    Q, K, V = W.make_qkv(wl)
+    orc = oracle.Layout(wl)
+    ref = oracle.forward(wl, Q, K, V, lay=orc)
+    lay = moc.Layout.from_workload(wl)
+    Qd, Kd, Vd = Q.cuda(), K.cuda(), V.cuda()
+    sel = torch.from_numpy(np.ascontiguousarray(ref["sel"])).cuda()
+    ws = moc.workspace(lay, wl.B, wl.H, wl.d, wl.k)
+    outs = []
+    try:
+        for n_ctas, rev in [(0, False), (5, True)]:
+            moc.set_attend_schedule(n_ctas, reverse=rev)
+            O = torch.empty_like(Qd)
+            lse = torch.empty(wl.B, wl.H, wl.L, dtype=torch.float32, device="cuda")
+            moc.build_qlists(lay, sel, wl.B, wl.H, wl.k, ws)
+            moc.attend_merged(lay, Qd, Kd, Vd, sel, wl.k, ws, O, lse)
+            torch.cuda.synchronize()
+            assert moc.check_device_error(ws) == 0
+            compare_attention(O.cpu(), lse.cpu(), ref["O"], ref["lse"])
+            outs.append((O.cpu(), lse.cpu()))
+    finally:
+        moc.set_attend_schedule(0, reverse=False)
+    assert torch.equal(outs[0][0].view(torch.int16), outs[1][0].view(torch.int16))
+    assert torch.equal(outs[0][1], outs[1][1])
