@@ -81,13 +81,29 @@ struct KUnit {
     int bh, blk, k0, nk, chunk;
 };
 
+// Units in order: the leading blocks (caption runs, attended by every query: the
+// longest units) block by block, each for every (b, h); then the video chunks'
+// blocks head by head, so that the units running at one time share one head's
+// query rows (a head's Q and dO stay in L2 while its chunks' units read them).
 __device__ __forceinline__ void decode_k(const DevLayout& dv, int BH, int64_t u, KUnit& x) {
-    const int pos = upper_index(dv.kt_off, dv.NKB + 1, u / BH);
-    const int64_t local = u - int64_t(BH) * dv.kt_off[pos];
-    const int nt = dv.kt_off[pos + 1] - dv.kt_off[pos];
+    const int64_t lead = int64_t(BH) * dv.kt_off[dv.kb_lead];
+    int pos, tile;
+    if (u < lead) {
+        pos = upper_index(dv.kt_off, dv.NKB + 1, u / BH);
+        const int64_t local = u - int64_t(BH) * dv.kt_off[pos];
+        const int nt = dv.kt_off[pos + 1] - dv.kt_off[pos];
+        x.bh = int(local / nt);
+        tile = int(local % nt);
+    } else {
+        const int64_t per_head = dv.kt_off[dv.NKB] - dv.kt_off[dv.kb_lead];
+        const int64_t r = u - lead;
+        x.bh = int(r / per_head);
+        const int64_t t = dv.kt_off[dv.kb_lead] + r % per_head;
+        pos = upper_index(dv.kt_off, dv.NKB + 1, t);
+        tile = int(t - dv.kt_off[pos]);
+    }
     x.blk = dv.kb_order[pos];
-    x.bh = int(local / nt);
-    x.k0 = dv.kb_range[2 * x.blk] + int(local % nt) * kQTile;
+    x.k0 = dv.kb_range[2 * x.blk] + tile * kQTile;
     x.nk = min(kQTile, dv.kb_range[2 * x.blk + 1] - x.k0);
     x.chunk = dv.kb_chunk[x.blk];
 }

@@ -250,6 +250,9 @@ moc_status build_host(const moc_layout_desc* d, moc_layout* lay) {
         lay->kt_off.push_back(lay->kt_off.back() + (nk + moc::kQTile - 1) / moc::kQTile);
     }
     lay->total_ktiles = lay->kt_off.back();
+    // caption runs are attended by every query (the longest units): they lead
+    lay->kb_lead = 0;
+    while (lay->kb_lead < NKB && lay->kb_chunk[lay->kb_order[lay->kb_lead]] < 0) ++lay->kb_lead;
     return MOC_OK;
 }
 
@@ -312,6 +315,7 @@ moc_status upload(moc_layout* lay) {
     dv.kb_grp = at(21);
     dv.kb_order = at(22);
     dv.kt_off = at(23);
+    dv.kb_lead = lay->kb_lead;
     dv.err = reinterpret_cast<int32_t*>(static_cast<char*>(lay->dev_block) + err_off);
     return MOC_OK;
 }

@@ -47,6 +47,7 @@ struct DevLayout {
     const int32_t* kb_grp;       // query groups whose anchor ranges hold the block
     const int32_t* kb_order;     // [NKB] blocks by descending anchoring query rows
     const int32_t* kt_off;       // [NKB+1] prefix of 128-key tiles over kb_order
+    int32_t kb_lead;             // leading blocks of kb_order handed out block-major (caption runs)
 };
 
 }  // namespace moc
@@ -66,6 +67,7 @@ struct moc_layout {
     std::vector<int64_t> grp_keys;  // anchor keys of each group
     std::vector<int32_t> kb_range, kb_chunk, kb_goff, kb_grp, kb_order, kt_off;  // backward key blocks
     int64_t total_ktiles = 0;       // 128-key tiles per (b, h)
+    int32_t kb_lead = 0;            // caption-run blocks at the head of kb_order
     void* dev_block = nullptr;
     moc::DevLayout dv{};
 };
