@@ -57,9 +57,9 @@ struct RWarps {
 
 // Shared memory of one CTA: a QS-stage ring of 128-row Q tiles and the hi / lo
 // operand blocks of KBLK candidates. Groups with at most 128 candidates (every
-// group of the eight-shot scene has <= 105) use KBLK = 128, which leaves room
-// for a deeper Q ring (more bytes in flight per SM); larger candidate lists use
-// KBLK = 256 and a 2-stage ring.
+// group of the eight-shot scene has <= 105) use KBLK = 128 with a 5-stage ring;
+// up to 320 candidates (the ragged and stress scenes) KBLK = 320 with a 2-stage
+// ring, so that a group's whole list sits in one block; larger lists KBLK = 256.
 template <int D, int KBLK, int QS>
 struct RCfg {
     static constexpr int kBlk = KBLK;                   // candidates per operand block
@@ -371,6 +371,15 @@ __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
                 continue;
             }
             const uint64_t smask = seg_mask ? seg_mask[size_t(x.bh) * dv.G + x.g] : ~0ull;
+            // with 128-row operand blocks every candidate list has <= 128 entries: the
+            // warp loads the group's chunk ids now (lane l holds entries l, l+32, ...),
+            // so the loads overlap the score wait and the ids are mapped with shuffles
+            int cid[4] = {-1, -1, -1, -1};
+            if (kBlk == 128) {
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+                    if (r * 32 + lane < x.ncand) cid[r] = __ldg(dv.cand + x.cbeg + r * 32 + lane);
+            }
             float ts[KMAX];
             int tj[KMAX];
 #pragma unroll
@@ -408,7 +417,17 @@ __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
                 ++u;
             }
             if (stop) break;
-            if (row < x.nq) {
+            if (kBlk == 128) {
+#pragma unroll
+                for (int j = 0; j < KMAX; ++j) {
+                    const int pos = tj[j] == kIdNone ? 0 : tj[j];
+                    const int src = pos & 31, r = pos >> 5;
+                    const int i0 = __shfl_sync(0xffffffffu, cid[0], src), i1 = __shfl_sync(0xffffffffu, cid[1], src);
+                    const int i2 = __shfl_sync(0xffffffffu, cid[2], src), i3 = __shfl_sync(0xffffffffu, cid[3], src);
+                    const int id = r == 0 ? i0 : r == 1 ? i1 : r == 2 ? i2 : i3;
+                    if (row < x.nq && j < k) out[size_t(row) * k + j] = (tj[j] == kIdNone) ? -1 : id;
+                }
+            } else if (row < x.nq) {
 #pragma unroll
                 for (int j = 0; j < KMAX; ++j)
                     if (j < k) out[size_t(row) * k + j] = (tj[j] == kIdNone) ? -1 : __ldg(dv.cand + x.cbeg + tj[j]);
@@ -444,9 +463,10 @@ cudaError_t launch_cfg(const DevLayout& dv, int BH, int64_t rtiles, const void* 
 }
 
 // Candidate lists of at most 128 entries fit one 128-row operand block, which
-// frees shared memory for a 5-stage Q ring; longer lists take 256-row blocks and
-// a 2-stage ring. (With 2 selection warpgroups a slice is 256 candidates, which
-// needs the 256-row block.)
+// frees shared memory for a 5-stage Q ring; lists of up to 320 entries take one
+// 320-row block and a 2-stage ring; longer lists take 256-row blocks (rebuilt as
+// a tile's slices cross them) and a 2-stage ring. (With 2 selection warpgroups a
+// slice is 256 candidates, which needs a block of at least 256 rows.)
 template <int D, int KMAX>
 cudaError_t launch_dk(const DevLayout& dv, int BH, int64_t rtiles, const void* Q, const float* Kbar, int k,
                       int causal, int max_cand, const uint64_t* seg_mask, int32_t* sel, cudaStream_t s) {
@@ -454,6 +474,10 @@ cudaError_t launch_dk(const DevLayout& dv, int BH, int64_t rtiles, const void* Q
         if (max_cand <= 128)
             return launch_cfg<D, KMAX, 128, 5>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
     }
+    // lists of up to 320 entries fit one operand block beside a 2-stage ring, so a
+    // group's block is built once instead of once per tile and block
+    if (max_cand <= 320)
+        return launch_cfg<D, KMAX, 320, 2>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
     return launch_cfg<D, KMAX, 256, 2>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
 }
 
