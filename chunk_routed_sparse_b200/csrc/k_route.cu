@@ -33,9 +33,6 @@
 //          (-1 padded) after the tile's last slice. The network is a chain of
 //          dependent compare/select steps per row, so more warpgroups (more
 //          rows in flight per scheduler) hide its latency.
-// Candidate lists of at most 128 entries with k <= 8 (the eight-shot scene) go
-// to route_ws_kernel below instead, where each selection warpgroup issues its
-// own MMAs.
 // Tiles without candidates (caption groups, the first shot) are written as -1
 // rows by their selection warpgroup and skip the other roles. Waits are
 // bounded as in the attention kernel; a timeout is recorded in the layout's
@@ -125,6 +122,27 @@ __device__ __forceinline__ void topk_push(float (&ts)[KMAX], int (&tj)[KMAX], fl
     }
 }
 
+// For k > 4: an order-preserving 32-bit key of a score with the candidate's
+// position in its 9 low bits (larger score first, then lower position), so an
+// insertion step is one max and one min. The score keeps all but the 9 lowest
+// bits of its order-preserving integer image: scores closer than 2^-14 of their
+// magnitude compare equal and go by position (chunk id), a gap well inside the
+// 1e-4 relative near-tie tolerance that routing is checked with.
+__device__ __forceinline__ uint32_t pack_key(float s, int pos) {
+    const uint32_t u = __float_as_uint(s);
+    const uint32_t o = u ^ (uint32_t(int32_t(u) >> 31) | 0x80000000u);
+    return (o & ~0x1FFu) | (0x1FFu - uint32_t(pos));
+}
+template <int KMAX>
+__device__ __forceinline__ void topk_push_key(uint32_t (&t)[KMAX], uint32_t c) {
+#pragma unroll
+    for (int x = 0; x < KMAX; ++x) {
+        const uint32_t hi = max(t[x], c);
+        c = min(t[x], c);
+        t[x] = hi;
+    }
+}
+
 struct Tile {
     int bh, g, q0, nq, cbeg, ncand, nb;
 };
@@ -211,7 +229,7 @@ __device__ __forceinline__ void build_block(const DevLayout& dv, const float* __
     }
 }
 
-template <int D, int KMAX, int KBLK, int QS>
+template <int D, int KMAX, int KBLK, int QS, bool PK>
 __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
     route_tc_kernel(const __grid_constant__ CUtensorMap tmQ, DevLayout dv, int64_t total_tiles,
                     int64_t rtiles, const float* __restrict__ Kbar, int k, int causal,
@@ -385,10 +403,12 @@ __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
             }
             float ts[KMAX];
             int tj[KMAX];
+            uint32_t tk[KMAX];
 #pragma unroll
             for (int j = 0; j < KMAX; ++j) {
                 ts[j] = -INFINITY;
                 tj[j] = kIdNone;
+                tk[j] = 0u;
             }
             bool stop = false;
             for (int b = 0; b < x.nb; ++b) {
@@ -412,14 +432,21 @@ __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
                         allow = __ballot_sync(0xffffffffu, ok);
                     }
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if ((allow >> e) & 1u) topk_push<KMAX>(ts, tj, __uint_as_float(sc[e]), pos0 + e);
+                    for (int e = 0; e < 32; ++e) {
+                        if (!((allow >> e) & 1u)) continue;
+                        if (PK) topk_push_key<KMAX>(tk, pack_key(__uint_as_float(sc[e]), pos0 + e));
+                        else topk_push<KMAX>(ts, tj, __uint_as_float(sc[e]), pos0 + e);
+                    }
                 }
                 tc_fence_before();
                 mbar_arrive(bar(R_S_FREE + w));
                 ++u;
             }
             if (stop) break;
+            if (PK) {
+#pragma unroll
+                for (int j = 0; j < KMAX; ++j) tj[j] = tk[j] == 0u ? kIdNone : int(0x1FFu - (tk[j] & 0x1FFu));
+            }
             if (kBlk == 128) {
 #pragma unroll
                 for (int j = 0; j < KMAX; ++j) {
@@ -446,315 +473,13 @@ __global__ void __launch_bounds__(RWarps<KMAX>::kThreads, 1)
     }
 }
 
-// ---------------------------------------------------------------------------
-// The router for candidate lists of at most 128 entries and k <= 8, with one
-// MMA issuer per selection warpgroup. A single issuing thread spends most of
-// the kernel issuing each tile's 16 MMAs and its per-tile bookkeeping, while
-// the selection warpgroups wait for scores; here every warpgroup issues its own
-// tiles' MMAs into its own 128-column TMEM slice, so four tiles' issue work
-// proceeds in parallel and the tensor pipe takes MMAs from four threads. The
-// hi / lo operand block of a (head, group) is built by a builder warp into one
-// of two buffers (block versions alternate), ahead of the tiles that use it: a
-// version's buffer is rebuilt only once every warpgroup has moved past the
-// version two before (its MMAs, waited for through its scores, are complete).
-template <int D>
-struct WsCfg {
-    static constexpr int kSlabs = D / 64;
-    static constexpr int kQBytes = kSlabs * 128 * 128;  // one 128-row Q tile
-    static constexpr int kKbSlab = 128 * 128;           // 128 candidate rows x 128 B
-    static constexpr int kKbBytes = kSlabs * kKbSlab;   // hi (or lo) block
-    static constexpr int kQStages = 3;
-    static constexpr int oQ = 0;
-    static constexpr int oBlk = oQ + kQStages * kQBytes;  // [version & 1][hi, lo]
-    static constexpr int oBar = oBlk + 2 * 2 * kKbBytes;
-    static constexpr int kSmem = (oBar + 512 + 1024) > 120 * 1024 ? (oBar + 512 + 1024) : 120 * 1024;
-    static_assert(kSmem <= 227 * 1024, "shared memory");
-};
-
-enum { W_Q_FULL = 0, W_Q_EMPTY = 4, W_S_FULL = 8, W_S_FREE = 12, W_DONE = 16 };
-
-struct WsShared {  // at oBar + 256
-    uint32_t tmem_base;
-    int abort;
-    int64_t t_beg, t_end;
-    int done_ver[4];  // every block version below this warpgroup's current tile's is done with
-    int ready_ver;    // highest block version built
-};
-
-__device__ __forceinline__ int ld_acquire_cta(const int* p) {
-    int v;
-    asm volatile("ld.acquire.cta.shared.b32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_release_cta(int* p, int v) {
-    asm volatile("st.release.cta.shared.b32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
-}
-
-// Block version of each tile with candidates: increments at every (head, group)
-// change along the walk (every role counts it the same way).
-struct VerCount {
-    int ver = -1, bh = -1, g = -1;
-    __device__ __forceinline__ int of(const Tile& x) {
-        if (x.bh != bh || x.g != g) {
-            ++ver;
-            bh = x.bh;
-            g = x.g;
-        }
-        return ver;
-    }
-};
-
-template <int D, int KMAX>
-__global__ void __launch_bounds__(576, 1)
-    route_ws_kernel(const __grid_constant__ CUtensorMap tmQ, DevLayout dv, int64_t total_tiles, int64_t rtiles,
-                    const float* __restrict__ Kbar, int k, int causal, const uint64_t* __restrict__ seg_mask,
-                    int32_t* __restrict__ sel) {
-    using C = WsCfg<D>;
-    constexpr int NWG = 4, SLICE = 128, QS = C::kQStages;
-    extern __shared__ __align__(1024) unsigned char smem_raw[];
-    const uint32_t raw = smem_u32(smem_raw);
-    const uint32_t base = (raw + 1023u) & ~1023u;
-    unsigned char* gbase = smem_raw + (base - raw);
-    const uint32_t sQ = base + C::oQ, sBlk = base + C::oBlk;
-    const uint32_t sBar = base + C::oBar;
-    WsShared& sh = *reinterpret_cast<WsShared*>(gbase + C::oBar + 256);
-    volatile int* abort = &sh.abort;
-    int32_t* err = dv.err;
-    auto bar = [&](int i) { return sBar + 8u * uint32_t(i); };
-    auto hi_of = [&](int v) { return sBlk + uint32_t(v & 1) * 2 * C::kKbBytes; };
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    constexpr int kProducer = 16, kBuilder = 17;
-
-    if (tid == 0) {
-        for (int x = 0; x < QS; ++x) {
-            mbar_init(bar(W_Q_FULL + x), 1);
-            mbar_init(bar(W_Q_EMPTY + x), 1);
-        }
-        for (int x = 0; x < NWG; ++x) {
-            mbar_init(bar(W_S_FULL + x), 1);
-            mbar_init(bar(W_S_FREE + x), 128);
-            mbar_init(bar(W_DONE + x), 1);
-            sh.done_ver[x] = -1;
-        }
-        sh.ready_ver = -1;
-        sh.abort = 0;
-        const int64_t total_cost = (total_tiles / rtiles) * int64_t(dv.rcost[causal ? 1 : 0][rtiles]);
-        sh.t_beg = tile_at_cost(dv, rtiles, causal, total_tiles, total_cost * blockIdx.x / gridDim.x);
-        sh.t_end = tile_at_cost(dv, rtiles, causal, total_tiles, total_cost * (blockIdx.x + 1) / gridDim.x);
-        fence_mbar_init();
-    }
-    if (warp == kBuilder) {
-        tmem_alloc(smem_u32(&sh.tmem_base), 512);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = sh.tmem_base;
-    const int64_t t_beg = sh.t_beg, t_end = sh.t_end;
-
-    if (warp == kProducer) {
-        // ------------------------------------------------------------ Q producer
-        if (lane == 0) {
-            prefetch_tmap(&tmQ);
-            uint32_t qi = 0;
-            TileWalk<SLICE> walk;
-            if (t_beg < t_end) walk.start(dv, rtiles, causal, t_beg);
-            for (int64_t t = t_beg; t < t_end; ++t, walk.advance(dv, rtiles, causal)) {
-                const Tile x = walk.tile();
-                if (x.ncand == 0) continue;
-                const int st = qi % QS;
-                if (!wait_bar(bar(W_Q_EMPTY + st), ((qi / QS) & 1) ^ 1, abort, err, 41)) break;
-                mbar_expect_tx(bar(W_Q_FULL + st), C::kQBytes);
-#pragma unroll
-                for (int s = 0; s < C::kSlabs; ++s)
-                    tma_load_2d(sQ + st * C::kQBytes + s * 128 * 128, &tmQ, bar(W_Q_FULL + st), 64 * s,
-                                x.bh * dv.L + x.q0);
-                ++qi;
-            }
-            for (uint32_t g = (qi >= uint32_t(QS) ? qi - QS : 0); g < qi; ++g)
-                drain_bar(bar(W_Q_FULL + g % QS), (g / QS) & 1, err, 42);
-        }
-        __syncwarp();
-    } else if (warp == kBuilder) {
-        // ------------------------------------------------------------ operand-block builder
-        VerCount vc;
-        TileWalk<SLICE> walk;
-        if (t_beg < t_end) walk.start(dv, rtiles, causal, t_beg);
-        for (int64_t t = t_beg; t < t_end; ++t, walk.advance(dv, rtiles, causal)) {
-            const Tile x = walk.tile();
-            if (x.ncand == 0) continue;
-            const int prev = vc.ver;
-            const int v = vc.of(x);
-            if (v == prev) continue;
-            // buffer v & 1 last held version v - 2: every warpgroup must be past it
-            bool ok = true;
-            if (lane == 0 && v >= 2) {
-                const uint64_t t0 = globaltimer();
-                for (;;) {
-                    int m = ld_acquire_cta(&sh.done_ver[0]);
-                    for (int w = 1; w < NWG; ++w) m = min(m, ld_acquire_cta(&sh.done_ver[w]));
-                    if (m >= v - 2) break;
-                    if (*abort) { ok = false; break; }
-                    if (globaltimer() - t0 > kTimeoutNs) { set_error(err, ERR_TIMEOUT, 43); *abort = 1; ok = false; break; }
-                }
-            }
-            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            const uint32_t hi = hi_of(v), lo = hi + C::kKbBytes;
-            build_block<D, C::kKbSlab, 128>(dv, Kbar, x.bh, x.cbeg, 0, x.ncand, (x.ncand + 15) & ~15, hi, lo, lane);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) st_release_cta(&sh.ready_ver, v);
-        }
-        __syncwarp();
-    } else if (warp < 4 * NWG) {
-        // ------------------------------------------------------------ selection warpgroups (each issues its MMAs)
-        const int wg = warp >> 2;
-        const int row = tid & 127;
-        const uint32_t lane_addr = tmem + (uint32_t((warp & 3) * 32) << 16) + wg * SLICE;
-        uint32_t u = 0, qi = 0;
-        int ti = 0;
-        VerCount vc;
-        TileWalk<SLICE> walk;
-        if (t_beg < t_end) walk.start(dv, rtiles, causal, t_beg);
-        for (int64_t t = t_beg; t < t_end; ++t, ++ti, walk.advance(dv, rtiles, causal)) {
-            const Tile x = walk.tile();
-            int v = -1, st = 0;
-            uint32_t ph = 0;
-            if (x.ncand > 0) {
-                v = vc.of(x);
-                st = int(qi % QS);
-                ph = (qi / QS) & 1;
-                ++qi;
-            }
-            if (ti % NWG != wg) continue;
-            int32_t* out = sel + (size_t(x.bh) * dv.L + x.q0) * k;
-            if (x.ncand == 0) {
-                if (row < x.nq)
-                    for (int j = 0; j < k; ++j) out[size_t(row) * k + j] = -1;
-                continue;
-            }
-            // every earlier tile of this warpgroup has its scores read: its block
-            // versions below v are done with
-            if (row == 0) st_release_cta(&sh.done_ver[wg], v - 1);
-            int cid[4];
-#pragma unroll
-            for (int r = 0; r < 4; ++r) cid[r] = (r * 32 + lane < x.ncand) ? __ldg(dv.cand + x.cbeg + r * 32 + lane) : -1;
-            const uint64_t smask = seg_mask ? seg_mask[size_t(x.bh) * dv.G + x.g] : ~0ull;
-            bool stop = false;
-            if ((warp & 3) == 0) {
-                // this warpgroup's issuing warp: Q tile landed, own slice free, block built
-                if (!wait_bar_warp(bar(W_Q_FULL + st), ph, abort, err, 44)) stop = true;
-                if (!stop && !wait_bar_warp(bar(W_S_FREE + wg), (u & 1) ^ 1, abort, err, 45)) stop = true;
-                if (!stop && lane == 0) {
-                    const uint64_t t0 = globaltimer();
-                    while (ld_acquire_cta(&sh.ready_ver) < v) {
-                        if (*abort) { stop = true; break; }
-                        if (globaltimer() - t0 > kTimeoutNs) { set_error(err, ERR_TIMEOUT, 46); *abort = 1; stop = true; break; }
-                    }
-                }
-                stop = __shfl_sync(0xffffffffu, stop, 0);
-                if (!stop) {
-                    tc_fence_after();
-                    if (lane == 0) {
-                        const int npad = (x.ncand + 15) & ~15;
-                        const uint32_t idesc = idesc_bf16_f32(128, npad, 0);
-                        const uint32_t hi = hi_of(v), lo = hi + C::kKbBytes;
-                        const uint64_t dq = sdesc_sw128(sQ + st * C::kQBytes, 16, 1024);
-                        const uint64_t dhi = sdesc_sw128(hi, 16, 1024), dlo = sdesc_sw128(lo, 16, 1024);
-#pragma unroll
-                        for (int kk = 0; kk < 2 * (D / 16); ++kk) {
-                            const int kd = kk % (D / 16);
-                            const uint32_t qoff = (kd >> 2) * 128 * 128 + (kd & 3) * 32;
-                            const uint32_t boff = (kd >> 2) * C::kKbSlab + (kd & 3) * 32;
-                            umma_ss(tmem + wg * SLICE, dq + (qoff >> 4), (kk < D / 16 ? dhi : dlo) + (boff >> 4), idesc,
-                                    kk > 0);
-                        }
-                        umma_commit(bar(W_S_FULL + wg));
-                        umma_commit(bar(W_Q_EMPTY + st));
-                    }
-                    __syncwarp();
-                }
-            }
-            if (stop) break;
-            float ts[KMAX];
-            int tj[KMAX];
-#pragma unroll
-            for (int j = 0; j < KMAX; ++j) {
-                ts[j] = -INFINITY;
-                tj[j] = kIdNone;
-            }
-            if (!wait_bar_warp(bar(W_S_FULL + wg), u & 1, abort, err, 47)) break;
-            tc_fence_after();
-            const int nbc = x.ncand;
-            for (int c0 = 0; c0 < nbc; c0 += 32) {
-                uint32_t sc[32];
-                tmem_ld32(lane_addr + c0, sc);
-                tmem_wait_ld_regs(sc);
-                uint32_t allow = (nbc - c0 >= 32) ? 0xffffffffu : ((1u << (nbc - c0)) - 1u);
-                if (seg_mask) {
-                    const bool okc = ((allow >> lane) & 1u) && ((smask >> dv.cand_seg[x.cbeg + c0 + lane]) & 1ull);
-                    allow = __ballot_sync(0xffffffffu, okc);
-                }
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    if ((allow >> e) & 1u) topk_push<KMAX>(ts, tj, __uint_as_float(sc[e]), c0 + e);
-            }
-            tc_fence_before();
-            mbar_arrive(bar(W_S_FREE + wg));
-            ++u;
-#pragma unroll
-            for (int j = 0; j < KMAX; ++j) {
-                const int pos = tj[j] == kIdNone ? 0 : tj[j];
-                const int src = pos & 31, r = pos >> 5;
-                const int i0 = __shfl_sync(0xffffffffu, cid[0], src), i1 = __shfl_sync(0xffffffffu, cid[1], src);
-                const int i2 = __shfl_sync(0xffffffffu, cid[2], src), i3 = __shfl_sync(0xffffffffu, cid[3], src);
-                const int id = r == 0 ? i0 : r == 1 ? i1 : r == 2 ? i2 : i3;
-                if (row < x.nq && j < k) out[size_t(row) * k + j] = (tj[j] == kIdNone) ? -1 : id;
-            }
-        }
-        // no further block version is needed by this warpgroup; every MMA it issued
-        // has completed before TMEM is released (a tile cut short by an abort may
-        // have issued MMAs whose scores were never waited for)
-        if (row == 0) {
-            st_release_cta(&sh.done_ver[wg], 0x7fffffff);
-            umma_commit(bar(W_DONE + wg));
-            drain_bar(bar(W_DONE + wg), 0, err, 48);
-        }
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    if (warp == kBuilder) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 512);
-    }
-}
-
-template <int D, int KMAX>
-cudaError_t launch_ws(const DevLayout& dv, int BH, int64_t rtiles, const void* Q, const float* Kbar, int k,
-                      int causal, const uint64_t* seg_mask, int32_t* sel, cudaStream_t s) {
-    CUtensorMap tmQ;
-    if (!make_tmap(&tmQ, Q, D, int64_t(BH) * dv.L)) return cudaErrorInvalidValue;
-    const int smem = WsCfg<D>::kSmem;
-    cudaError_t e = cudaFuncSetAttribute(route_ws_kernel<D, KMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t total = int64_t(BH) * rtiles;
-    const int grid = int(total < sms ? total : sms);
-    route_ws_kernel<D, KMAX><<<grid, 576, smem, s>>>(tmQ, dv, total, rtiles, Kbar, k, causal, seg_mask, sel);
-    return cudaGetLastError();
-}
-
-template <int D, int KMAX, int KBLK, int QS>
+template <int D, int KMAX, int KBLK, int QS, bool PK>
 cudaError_t launch_cfg(const DevLayout& dv, int BH, int64_t rtiles, const void* Q, const float* Kbar, int k,
                        int causal, const uint64_t* seg_mask, int32_t* sel, cudaStream_t s) {
     CUtensorMap tmQ;
     if (!make_tmap(&tmQ, Q, D, int64_t(BH) * dv.L)) return cudaErrorInvalidValue;
     const int smem = RCfg<D, KBLK, QS>::kSmem;
-    cudaError_t e = cudaFuncSetAttribute(route_tc_kernel<D, KMAX, KBLK, QS>,
+    cudaError_t e = cudaFuncSetAttribute(route_tc_kernel<D, KMAX, KBLK, QS, PK>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
@@ -762,8 +487,8 @@ cudaError_t launch_cfg(const DevLayout& dv, int BH, int64_t rtiles, const void* 
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t total = int64_t(BH) * rtiles;
     const int grid = int(total < sms ? total : sms);
-    route_tc_kernel<D, KMAX, KBLK, QS><<<grid, RWarps<KMAX>::kThreads, smem, s>>>(tmQ, dv, total, rtiles, Kbar, k,
-                                                                                  causal, seg_mask, sel);
+    route_tc_kernel<D, KMAX, KBLK, QS, PK><<<grid, RWarps<KMAX>::kThreads, smem, s>>>(tmQ, dv, total, rtiles, Kbar,
+                                                                                      k, causal, seg_mask, sel);
     return cudaGetLastError();
 }
 
@@ -776,13 +501,22 @@ template <int D, int KMAX>
 cudaError_t launch_dk(const DevLayout& dv, int BH, int64_t rtiles, const void* Q, const float* Kbar, int k,
                       int causal, int max_cand, const uint64_t* seg_mask, int32_t* sel, cudaStream_t s) {
     if constexpr (RWarps<KMAX>::kSlice <= 128) {
-        if (max_cand <= 128) return launch_ws<D, KMAX>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
+        if (max_cand <= 128)
+            return launch_cfg<D, KMAX, 128, 5, (KMAX >= 8)>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
     }
     // lists of up to 320 entries fit one operand block beside a 2-stage ring, so a
-    // group's block is built once instead of once per tile and block
-    if (max_cand <= 320)
-        return launch_cfg<D, KMAX, 320, 2>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
-    return launch_cfg<D, KMAX, 256, 2>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
+    // group's block is built once instead of once per tile and block; for k > 4
+    // the selection uses packed score / position keys (positions below 512)
+    if constexpr (KMAX >= 8) {
+        if (max_cand <= 320)
+            return launch_cfg<D, KMAX, 320, 2, true>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
+        if (max_cand <= 511)
+            return launch_cfg<D, KMAX, 256, 2, true>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
+    } else {
+        if (max_cand <= 320)
+            return launch_cfg<D, KMAX, 320, 2, false>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
+    }
+    return launch_cfg<D, KMAX, 256, 2, false>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
 }
 
 template <int D>
