@@ -65,6 +65,9 @@ SIGNATURES = {
     "moc_attend_partials": (_I, [_P, _I, _I, _I, _P, _P, _P, _I, _F, _P, _SZ, _P]),
     "moc_merge": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _SZ, _P]),
     "moc_attend_merged": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _F, _P, _P, _P, _SZ, _P]),
+    "moc_quantize_e4m3": (_I, [_I, _I64, _I, _P, _P, _P, _P]),
+    "moc_attend_partials_e4m3": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _I, _F, _P, _SZ, _P]),
+    "moc_attention_fwd_e4m3": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _I, _F, _P, _P, _P, _SZ, _P]),
     "moc_attention_fwd": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _F, _P, _P, _P, _SZ, _P]),
     "moc_attention_fwd_static": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _F, _P, _P, _P]),
     "moc_attention_bwd_workspace_bytes": (_SZ, [_P, _I, _I, _I, _I]),
@@ -330,6 +333,35 @@ def forward(layout: Layout, Q, K, V, k: int, causal: bool = True, scale=None, ws
         torch.empty(Q.shape[0], Q.shape[1], Q.shape[2], 0, dtype=torch.int32, device=Q.device)
     O, lse = attention_fwd(layout, Q, K, V, sel, k, scale=scale, ws=ws)
     return O, lse, sel, kbar
+
+
+def quantize_e4m3(X: torch.Tensor):
+    """Per-(b, h) power-of-two scale and E4M3 bytes of a bf16 [B, H, L, d] tensor
+    (moc_quantize_e4m3). Returns (X8 uint8 [B, H, L, d], scale fp32 [B, H])."""
+    B, H, L, d = _dims(X)
+    X8 = torch.empty(B, H, L, d, dtype=torch.uint8, device=X.device)
+    scale = torch.empty(B, H, dtype=torch.float32, device=X.device)
+    _check(lib().moc_quantize_e4m3(B * H, L, d, _ptr(X), _ptr(X8), _ptr(scale), _stream()), "moc_quantize_e4m3")
+    return X8, scale
+
+
+def attention_fwd_e4m3(layout: Layout, Q8, K8, V8, q_scale, k_scale, v_scale, sel, k: int,
+                       scale: Optional[float] = None, ws: Optional[torch.Tensor] = None,
+                       O: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None):
+    """The attention stage on E4M3 inputs (moc_attention_fwd_e4m3); bf16 O, fp32 lse."""
+    B, H, L, d = Q8.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if ws is None:
+        ws = workspace(layout, B, H, d, k, Q8.device)
+    if O is None:
+        O = torch.empty(B, H, L, d, dtype=torch.bfloat16, device=Q8.device)
+    if lse is None:
+        lse = torch.empty(B, H, L, dtype=torch.float32, device=Q8.device)
+    _check(lib().moc_attention_fwd_e4m3(layout.handle, B, H, d, _ptr(Q8), _ptr(K8), _ptr(V8), _ptr(q_scale),
+                                        _ptr(k_scale), _ptr(v_scale), _ptr(sel) if k > 0 else None, k,
+                                        float(scale), _ptr(O), _ptr(lse), _ptr(ws), ws.numel(), _stream()),
+           "moc_attention_fwd_e4m3")
+    return O, lse
 
 
 def forward_host_device_bytes(layout: Layout, B: int, H: int, d: int, k: int, heads_per_chunk: int = 0) -> int:

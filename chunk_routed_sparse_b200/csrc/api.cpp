@@ -333,3 +333,44 @@ extern "C" moc_status moc_attention_bwd(const moc_layout* lay, int B, int H, int
     if (e == cudaSuccess) e = moc::launch_bwd_dkv(lay->dv, BH, d, Q, K, V, dO, lse, scale, w, p, dK, dV, s);
     return cuda_status(e);
 }
+
+extern "C" moc_status moc_quantize_e4m3(int BH, int64_t L, int d, const void* X, void* X8, float* scale,
+                                        moc_stream_t stream) {
+    if (BH < 0 || L < 0 || (d != 64 && d != 128)) return MOC_ERR_INVALID_ARG;
+    if (BH == 0 || L == 0) return MOC_OK;
+    if (!X || !X8 || !scale || !aligned16(X) || !aligned16(X8) || (reinterpret_cast<uintptr_t>(scale) & 3))
+        return MOC_ERR_INVALID_ARG;
+    return cuda_status(moc::launch_quant_e4m3(BH, L, d, X, X8, scale, (cudaStream_t)stream));
+}
+
+extern "C" moc_status moc_attend_partials_e4m3(const moc_layout* lay, int B, int H, int d, const void* Q8,
+                                               const void* K8, const void* V8, const float* q_scale,
+                                               const float* k_scale, const float* v_scale, int k, float scale,
+                                               void* ws, size_t ws_bytes, moc_stream_t stream) {
+    moc_status st = check_common(lay, B, H, d, k);
+    if (st != MOC_OK) return st;
+    if (d != 128) return MOC_ERR_UNSUPPORTED;
+    if (B * H == 0) return MOC_OK;
+    moc::WsPlan p;
+    if ((st = check_ws(lay, B, H, d, k, ws, ws_bytes, &p)) != MOC_OK) return st;
+    if (!Q8 || !K8 || !V8 || !aligned16(Q8) || !aligned16(K8) || !aligned16(V8)) return MOC_ERR_INVALID_ARG;
+    for (const float* t : {q_scale, k_scale, v_scale})
+        if (!t || (reinterpret_cast<uintptr_t>(t) & 3)) return MOC_ERR_INVALID_ARG;
+    if (!(scale > 0.0f) || scale != scale) return MOC_ERR_INVALID_ARG;
+    const int64_t n_anchor = int64_t(B) * H * lay->total_atiles;
+    return cuda_status(moc::launch_attend_e4m3(lay->dv, B * H, Q8, K8, V8, q_scale, k_scale, v_scale, k, scale,
+                                               n_anchor, static_cast<char*>(ws), p, (cudaStream_t)stream));
+}
+
+extern "C" moc_status moc_attention_fwd_e4m3(const moc_layout* lay, int B, int H, int d, const void* Q8,
+                                             const void* K8, const void* V8, const float* q_scale,
+                                             const float* k_scale, const float* v_scale, const int32_t* sel, int k,
+                                             float scale, void* O, float* lse, void* ws, size_t ws_bytes,
+                                             moc_stream_t stream) {
+    moc_status st;
+    if ((st = moc_build_qlists(lay, B, H, k, sel, ws, ws_bytes, stream)) != MOC_OK) return st;
+    if ((st = moc_attend_partials_e4m3(lay, B, H, d, Q8, K8, V8, q_scale, k_scale, v_scale, k, scale, ws,
+                                       ws_bytes, stream)) != MOC_OK)
+        return st;
+    return moc_merge(lay, B, H, d, k, sel, O, lse, ws, ws_bytes, stream);
+}

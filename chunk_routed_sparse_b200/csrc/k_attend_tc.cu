@@ -64,9 +64,14 @@ constexpr int kRegsSoftmax = 216;
 constexpr int kRegsOther = 72;
 constexpr uint32_t kTmemCols = 512;
 
-template <int D>
+// F8: Q, K, V in E4M3 (one byte an element; d = 128 only) and P written to TMEM
+// as E4M3, every MMA of kind::f8f6f4 (K = 32 elements an instruction).
+template <int D, bool F8>
 struct Cfg {
-    static constexpr int kSlabs = D / 64;                   // 128-byte slabs per row
+    static_assert(!F8 || D == 128, "the E4M3 path is built for d = 128");
+    static constexpr int kEB = F8 ? 1 : 2;                  // bytes per element
+    static constexpr int kKStep = F8 ? 32 : 16;             // K elements per MMA
+    static constexpr int kSlabs = D * kEB / 128;            // 128-byte slabs per row
     static constexpr int kSlabBytes = 128 * 128;            // 128 rows x 128 B
     static constexpr int kTileBytes = kSlabs * kSlabBytes;  // a 128-row Q, K or V tile
     static constexpr int oQ = 0;                            // Q_A, Q_B
@@ -75,8 +80,13 @@ struct Cfg {
     static constexpr int oBar = oV + 2 * kTileBytes;
     // + 1024 B alignment slack; at least 120 KB so that one CTA owns an SM (and its TMEM)
     static constexpr int kSmem = (oBar + 256 + 1024) > 120 * 1024 ? (oBar + 256 + 1024) : 120 * 1024;
-    static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, kKT, 0);
-    static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 1);
+    static constexpr uint32_t kIdescQK = F8 ? idesc_e4m3_f32(128, kKT, 0) : idesc_bf16_f32(128, kKT, 0);
+    static constexpr uint32_t kIdescPV = F8 ? idesc_e4m3_f32(128, D, 1) : idesc_bf16_f32(128, D, 1);
+    // E4M3 P carries a factor 2^6 (and O is rescaled once the row max grows by more
+    // than 2^2), so P * 64 <= 256 stays below E4M3's 448 and small weights stay
+    // normal numbers longer
+    static constexpr float kPScale = F8 ? 64.f : 1.f;
+    static constexpr float kLazy = F8 ? 2.f : 8.f;
 };
 
 // TMEM columns: S_A / S_B (P_A / P_B overwrite their first 64 columns), O_A / O_B
@@ -101,16 +111,19 @@ struct Shared {  // at oBar + 192
 // and writes the bf16 output row and its log-sum-exp (the merge of (5) done in
 // place, so slot 0 is never written and read back). Not FUSED: every item writes
 // its partial, for the stage call of (4) followed by (5).
-template <int D, bool FUSED>
+template <int D, bool FUSED, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      DevLayout dv, int BH, int k, float scale_log2, int64_t n_anchor,
-                     const __nv_bfloat16* __restrict__ Q, int32_t* __restrict__ hdr,
+                     const unsigned char* __restrict__ Q, int32_t* __restrict__ hdr,
                      const int32_t* __restrict__ qoff, const int32_t* __restrict__ tile_off,
                      const int32_t* __restrict__ qlist, float* __restrict__ lse_p,
                      float* __restrict__ o_p, int reverse, const int32_t* __restrict__ sel,
-                     __nv_bfloat16* __restrict__ O_out, float* __restrict__ lse_out) {
-    using C = Cfg<D>;
+                     __nv_bfloat16* __restrict__ O_out, float* __restrict__ lse_out,
+                     const float* __restrict__ q_scale, const float* __restrict__ k_scale,
+                     const float* __restrict__ v_scale) {
+    using C = Cfg<D, F8>;
+    static_assert(!(FUSED && F8), "the fused merge is built for bf16 inputs");
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // 1024-byte aligned base: the 128-byte swizzle atoms of TMA and UMMA repeat every 1024 B
     const uint32_t raw = smem_u32(smem_raw);
@@ -250,10 +263,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (!wait_bar(bar(B_P_FULL + q), g & 1, abort, hdr, 7)) { stop = true; break; }
                             tc_fence_after();
 #pragma unroll
-                            for (int kk = 0; kk < kKT / 16; ++kk)
-                                umma_ts(tmem + col_o(q), tmem + col_s(q) + kk * 8,
-                                        sdesc_sw128(sV + pst * C::kTileBytes + kk * 2048, C::kSlabBytes, 1024),
-                                        C::kIdescPV, (j > 1 || kk > 0));
+                            for (int kk = 0; kk < kKT / C::kKStep; ++kk) {
+                                // P's K step kk: 8 TMEM columns (16 bf16 or 32 E4M3 keys); V's: kKStep rows
+                                const uint64_t vd = sdesc_sw128(sV + pst * C::kTileBytes + kk * C::kKStep * 128,
+                                                                C::kSlabBytes, 1024);
+                                if constexpr (F8)
+                                    umma_ts_f8(tmem + col_o(q), tmem + col_s(q) + kk * 8, vd, C::kIdescPV, (j > 1 || kk > 0));
+                                else
+                                    umma_ts(tmem + col_o(q), tmem + col_s(q) + kk * 8, vd, C::kIdescPV, (j > 1 || kk > 0));
+                            }
                             umma_commit(bar(B_PV_DONE + q));
                         }
                         if (j < T) {  // S_q(j) = Q_q K(j)^T, after PV_q(j-1) has read P_q(j-1)
@@ -264,10 +282,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                             const uint32_t qb = sQ + q * C::kTileBytes, kb = sK + st * C::kTileBytes;
 #pragma unroll
-                            for (int kk = 0; kk < D / 16; ++kk) {
+                            for (int kk = 0; kk < D / C::kKStep; ++kk) {
+                                // 32 bytes of every row per K step in both element types
                                 const uint32_t off = (kk >> 2) * C::kSlabBytes + (kk & 3) * 32;
-                                umma_ss(tmem + col_s(q), sdesc_sw128(qb + off, 16, 1024),
-                                        sdesc_sw128(kb + off, 16, 1024), C::kIdescQK, kk > 0);
+                                if constexpr (F8)
+                                    umma_ss_f8(tmem + col_s(q), sdesc_sw128(qb + off, 16, 1024),
+                                               sdesc_sw128(kb + off, 16, 1024), C::kIdescQK, kk > 0);
+                                else
+                                    umma_ss(tmem + col_s(q), sdesc_sw128(qb + off, 16, 1024),
+                                            sdesc_sw128(kb + off, 16, 1024), C::kIdescQK, kk > 0);
                             }
                             umma_commit(bar(B_S_FULL + q));
                             ++gtt[q];
@@ -308,7 +331,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             decode(dv, BH, n_anchor, item, tile_off, qoff, qlist, itm);
             if (q == 1 && itm.nq <= kQTile) continue;  // no tile B in this item
             const int r_item = q * kQTile + row;       // row within the item
-            const __nv_bfloat16* Qb = Q + size_t(itm.bh) * L * D;
+            const unsigned char* Qb = Q + size_t(itm.bh) * L * D * C::kEB;
+            // scores are q . k in the inputs' units; E4M3 inputs carry per-(b, h) scales
+            const float sl2 = F8 ? scale_log2 * q_scale[itm.bh] * k_scale[itm.bh] : scale_log2;
             int my_tok = -1, my_slot = 0;
             if (r_item < itm.nq) {
                 if (itm.slot_fixed >= 0) {
@@ -322,13 +347,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             // gather the warp's 32 query rows into the swizzled tile (16-byte chunks):
             // every load is issued before the first store, so the warp waits for
             // one memory round trip instead of one per chunk
-            constexpr int CH = D / 8;
+            constexpr int CH = D * C::kEB / 16;
             uint4 qv[CH];
 #pragma unroll
             for (int i = 0; i < CH; ++i) {
                 const int tok = __shfl_sync(0xffffffffu, my_tok, (i * 32 + lane) / CH);
                 qv[i] = make_uint4(0, 0, 0, 0);
-                if (tok >= 0) qv[i] = ldg_nc16(Qb + size_t(tok) * D + ((i * 32 + lane) % CH) * 8);
+                if (tok >= 0) qv[i] = ldg_nc16(Qb + size_t(tok) * D * C::kEB + ((i * 32 + lane) % CH) * 16);
             }
 #pragma unroll
             for (int i = 0; i < CH; ++i) {
@@ -371,12 +396,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int i = 0; i < 8; ++i) a[i] = max3(a[i], __uint_as_float(s[c + 2 * i]), __uint_as_float(s[c + 2 * i + 1]));
                 }
-                const float mx = max3(max3(a[0], a[1], a[2]), max3(a[3], a[4], a[5]), fmaxf(a[6], a[7])) * scale_log2;
+                const float mx = max3(max3(a[0], a[1], a[2]), max3(a[3], a[4], a[5]), fmaxf(a[6], a[7])) * sl2;
                 float alpha = 1.f;
                 bool rescale = false;
                 if (j == 0) {
                     m_used = mx;
-                } else if (mx > m_used + 8.f) {  // lazy rescale: only when the max grew by > 2^8
+                } else if (mx > m_used + C::kLazy) {  // lazy rescale: only when the max grew by > 2^8 (E4M3: 2^2)
                     alpha = ex2(m_used - mx);
                     m_used = mx;
                     rescale = true;
@@ -397,22 +422,40 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 // P = exp2(s * scale - m) as bf16 pairs into the first 64 columns of S_q;
                 // scale-and-subtract and the row sum run on packed fp32 pairs
-                const uint64_t sc2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m_used, -m_used);
+                const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(-m_used, -m_used);
                 uint64_t sum2a = 0, sum2b = 0;
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
+                if constexpr (F8) {
+                    // four keys a column: E4M3 of P * 2^6 in the first 32 columns of S_q
                     uint32_t pk[32];
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
-                        const int e = h * 64 + 2 * c;
-                        float x0, x1;
+                        const int e = 4 * c;
+                        float x0, x1, x2, x3;
                         f2_unpack(f2_fma(f2_pack(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), sc2, nm2), x0, x1);
-                        const float p0 = ex2(x0), p1 = ex2(x1);
-                        if (c & 1) sum2b = f2_add(sum2b, f2_pack(p0, p1));
-                        else sum2a = f2_add(sum2a, f2_pack(p0, p1));
-                        pk[c] = pack_bf16(p0, p1);
+                        f2_unpack(f2_fma(f2_pack(__uint_as_float(s[e + 2]), __uint_as_float(s[e + 3])), sc2, nm2), x2, x3);
+                        const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
+                        sum2a = f2_add(sum2a, f2_pack(p0, p1));
+                        sum2b = f2_add(sum2b, f2_pack(p2, p3));
+                        pk[c] = pack_e4m3x2(p0 * C::kPScale, p1 * C::kPScale) |
+                                (pack_e4m3x2(p2 * C::kPScale, p3 * C::kPScale) << 16);
                     }
-                    tmem_st32(s_addr + h * 32, pk);
+                    tmem_st32(s_addr, pk);
+                } else {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t pk[32];
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            const int e = h * 64 + 2 * c;
+                            float x0, x1;
+                            f2_unpack(f2_fma(f2_pack(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), sc2, nm2), x0, x1);
+                            const float p0 = ex2(x0), p1 = ex2(x1);
+                            if (c & 1) sum2b = f2_add(sum2b, f2_pack(p0, p1));
+                            else sum2a = f2_add(sum2a, f2_pack(p0, p1));
+                            pk[c] = pack_bf16(p0, p1);
+                        }
+                        tmem_st32(s_addr + h * 32, pk);
+                    }
                 }
                 float r0, r1, r2, r3;
                 f2_unpack(sum2a, r0, r1);
@@ -499,7 +542,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (my_tok >= 0 && lse_out) lse_out[row] = M + logf(Z);
                 continue;
             }
-            const float inv = 1.f / l;
+            // E4M3: O accumulates P * 2^6 times the unscaled V
+            const float inv = F8 ? v_scale[itm.bh] / (C::kPScale * l) : 1.f / l;
             float* dst = (my_tok >= 0) ? o_p + ((size_t(itm.bh) * L + my_tok) * S + my_slot) * D : nullptr;
             float* rdst[8];  // destination row of this lane in store step i: row 4i + lane / 8
 #pragma unroll
@@ -555,15 +599,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int D, bool FUSED>
+template <int D, bool FUSED, bool F8>
 cudaError_t launch_d(const DevLayout& dv, int BH, const void* Q, const void* K, const void* V, int k,
                      float scale, int64_t n_anchor, char* ws, const WsPlan& p, const int32_t* sel, void* O,
-                     float* lse, cudaStream_t s) {
+                     float* lse, const float* q_scale, const float* k_scale, const float* v_scale,
+                     cudaStream_t s) {
     CUtensorMap tmK, tmV;
     const int64_t rows = int64_t(BH) * dv.L;
-    if (!make_tmap(&tmK, K, D, rows) || !make_tmap(&tmV, V, D, rows)) return cudaErrorInvalidValue;
-    const int smem = Cfg<D>::kSmem;
-    cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel<D, FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (F8) {
+        if (!make_tmap_u8(&tmK, K, D, rows) || !make_tmap_u8(&tmV, V, D, rows)) return cudaErrorInvalidValue;
+    } else {
+        if (!make_tmap(&tmK, K, D, rows) || !make_tmap(&tmV, V, D, rows)) return cudaErrorInvalidValue;
+    }
+    const int smem = Cfg<D, F8>::kSmem;
+    cudaError_t e =
+        cudaFuncSetAttribute(attend_tc_kernel<D, FUSED, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -573,11 +623,12 @@ cudaError_t launch_d(const DevLayout& dv, int BH, const void* Q, const void* K, 
     int32_t* hdr = reinterpret_cast<int32_t*>(ws + p.hdr);
     e = cudaMemsetAsync(hdr + HDR_WORK, 0, 2 * sizeof(int32_t), s);  // work counter, routed rows done
     if (e != cudaSuccess) return e;
-    attend_tc_kernel<D, FUSED><<<sms, kThreads, smem, s>>>(
-        tmK, tmV, dv, BH, k, scale * 1.4426950408889634f, n_anchor, static_cast<const __nv_bfloat16*>(Q), hdr,
+    attend_tc_kernel<D, FUSED, F8><<<sms, kThreads, smem, s>>>(
+        tmK, tmV, dv, BH, k, scale * 1.4426950408889634f, n_anchor, static_cast<const unsigned char*>(Q), hdr,
         reinterpret_cast<const int32_t*>(ws + p.qoff), reinterpret_cast<const int32_t*>(ws + p.tile_off),
         reinterpret_cast<const int32_t*>(ws + p.qlist), reinterpret_cast<float*>(ws + p.lse_p),
-        reinterpret_cast<float*>(ws + p.o_p), sched.reverse, sel, static_cast<__nv_bfloat16*>(O), lse);
+        reinterpret_cast<float*>(ws + p.o_p), sched.reverse, sel, static_cast<__nv_bfloat16*>(O), lse, q_scale,
+        k_scale, v_scale);
     return cudaGetLastError();
 }
 
@@ -586,15 +637,28 @@ cudaError_t launch_d(const DevLayout& dv, int BH, const void* Q, const void* K, 
 cudaError_t launch_attend_tc(const DevLayout& dv, int BH, int d, const void* Q, const void* K,
                              const void* V, int k, float scale, int64_t n_anchor, char* ws,
                              const WsPlan& p, cudaStream_t s) {
-    if (d == 128) return launch_d<128, false>(dv, BH, Q, K, V, k, scale, n_anchor, ws, p, nullptr, nullptr, nullptr, s);
-    return launch_d<64, false>(dv, BH, Q, K, V, k, scale, n_anchor, ws, p, nullptr, nullptr, nullptr, s);
+    if (d == 128)
+        return launch_d<128, false, false>(dv, BH, Q, K, V, k, scale, n_anchor, ws, p, nullptr, nullptr, nullptr,
+                                           nullptr, nullptr, nullptr, s);
+    return launch_d<64, false, false>(dv, BH, Q, K, V, k, scale, n_anchor, ws, p, nullptr, nullptr, nullptr, nullptr,
+                                      nullptr, nullptr, s);
 }
 
 cudaError_t launch_attend_merged(const DevLayout& dv, int BH, int d, const void* Q, const void* K,
                                  const void* V, int k, float scale, int64_t n_anchor, char* ws,
                                  const WsPlan& p, const int32_t* sel, void* O, float* lse, cudaStream_t s) {
-    if (d == 128) return launch_d<128, true>(dv, BH, Q, K, V, k, scale, n_anchor, ws, p, sel, O, lse, s);
-    return launch_d<64, true>(dv, BH, Q, K, V, k, scale, n_anchor, ws, p, sel, O, lse, s);
+    if (d == 128)
+        return launch_d<128, true, false>(dv, BH, Q, K, V, k, scale, n_anchor, ws, p, sel, O, lse, nullptr, nullptr,
+                                          nullptr, s);
+    return launch_d<64, true, false>(dv, BH, Q, K, V, k, scale, n_anchor, ws, p, sel, O, lse, nullptr, nullptr,
+                                     nullptr, s);
+}
+
+cudaError_t launch_attend_e4m3(const DevLayout& dv, int BH, const void* Q8, const void* K8, const void* V8,
+                               const float* q_scale, const float* k_scale, const float* v_scale, int k, float scale,
+                               int64_t n_anchor, char* ws, const WsPlan& p, cudaStream_t s) {
+    return launch_d<128, false, true>(dv, BH, Q8, K8, V8, k, scale, n_anchor, ws, p, nullptr, nullptr, nullptr,
+                                      q_scale, k_scale, v_scale, s);
 }
 
 }  // namespace moc

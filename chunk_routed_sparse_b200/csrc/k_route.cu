@@ -202,30 +202,46 @@ __device__ __forceinline__ void build_block(const DevLayout& dv, const float* __
                                             int b, int nbc, int npad, uint32_t sHi, uint32_t sLo, int lane) {
     const float* kb = Kbar + size_t(bh) * dv.C * D;
     constexpr int CH = D / 8;  // 16-byte output chunks (8 dims) per row
-    for (int i = lane; i < npad * CH; i += 32) {
-        const int r = i / CH, ch = i % CH;
-        float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        if (r < nbc) {
-            const int c = dv.cand[cbeg + b * KBLK + r];
-            const float4 a = *reinterpret_cast<const float4*>(kb + size_t(c) * D + ch * 8);
-            const float4 bq = *reinterpret_cast<const float4*>(kb + size_t(c) * D + ch * 8 + 4);
-            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-            v[4] = bq.x; v[5] = bq.y; v[6] = bq.z; v[7] = bq.w;
-        }
-        uint32_t hi[4], lo[4];
+    constexpr int U = 4;       // chunks per lane in flight: the id and Kbar loads of U chunks before their stores
+    const int n = npad * CH;
+    for (int i0 = lane; i0 < n; i0 += 32 * U) {
+        int cid[U];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
-            const float2 hf = __bfloat1622float2(h);
-            const __nv_bfloat162 l2 = __floats2bfloat162_rn(v[2 * e] - hf.x, v[2 * e + 1] - hf.y);
-            hi[e] = *reinterpret_cast<const uint32_t*>(&h);
-            lo[e] = *reinterpret_cast<const uint32_t*>(&l2);
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + 32 * u, r = i / CH;
+            cid[u] = (i < n && r < nbc) ? dv.cand[cbeg + b * KBLK + r] : -1;
         }
-        const uint32_t off = (ch >> 3) * KBSLAB + r * 128 + (((ch & 7) ^ (r & 7)) << 4);
-        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(sHi + off), "r"(hi[0]), "r"(hi[1]),
-                     "r"(hi[2]), "r"(hi[3]) : "memory");
-        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(sLo + off), "r"(lo[0]), "r"(lo[1]),
-                     "r"(lo[2]), "r"(lo[3]) : "memory");
+        float4 va[U], vb[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            va[u] = vb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (cid[u] >= 0) {
+                const int ch = (i0 + 32 * u) % CH;
+                va[u] = *reinterpret_cast<const float4*>(kb + size_t(cid[u]) * D + ch * 8);
+                vb[u] = *reinterpret_cast<const float4*>(kb + size_t(cid[u]) * D + ch * 8 + 4);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + 32 * u;
+            if (i >= n) break;
+            const int r = i / CH, ch = i % CH;
+            const float v[8] = {va[u].x, va[u].y, va[u].z, va[u].w, vb[u].x, vb[u].y, vb[u].z, vb[u].w};
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+                const float2 hf = __bfloat1622float2(h);
+                const __nv_bfloat162 l2 = __floats2bfloat162_rn(v[2 * e] - hf.x, v[2 * e + 1] - hf.y);
+                hi[e] = *reinterpret_cast<const uint32_t*>(&h);
+                lo[e] = *reinterpret_cast<const uint32_t*>(&l2);
+            }
+            const uint32_t off = (ch >> 3) * KBSLAB + r * 128 + (((ch & 7) ^ (r & 7)) << 4);
+            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(sHi + off), "r"(hi[0]), "r"(hi[1]),
+                         "r"(hi[2]), "r"(hi[3]) : "memory");
+            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(sLo + off), "r"(lo[0]), "r"(lo[1]),
+                         "r"(lo[2]), "r"(lo[3]) : "memory");
+        }
     }
 }
 

@@ -116,6 +116,10 @@ cudaError_t launch_attend_tc(const DevLayout& dv, int BH, int d, const void* Q, 
 cudaError_t launch_attend_merged(const DevLayout& dv, int BH, int d, const void* Q, const void* K,
                                  const void* V, int k, float scale, int64_t n_anchor, char* ws,
                                  const WsPlan& p, const int32_t* sel, void* O, float* lse, cudaStream_t s);
+cudaError_t launch_attend_e4m3(const DevLayout& dv, int BH, const void* Q8, const void* K8, const void* V8,
+                               const float* q_scale, const float* k_scale, const float* v_scale, int k, float scale,
+                               int64_t n_anchor, char* ws, const WsPlan& p, cudaStream_t s);
+cudaError_t launch_quant_e4m3(int BH, int64_t L, int d, const void* X, void* X8, float* scale, cudaStream_t s);
 cudaError_t launch_merge(int BH, int L, int d, int k, const int32_t* sel, void* O, float* lse,
                          const char* ws, const WsPlan& p, cudaStream_t s);
 

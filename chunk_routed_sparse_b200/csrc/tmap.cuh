@@ -38,4 +38,18 @@ static inline bool make_tmap(CUtensorMap* tm, const void* ptr, int d, int64_t ro
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [rows][row_bytes] one-byte elements (E4M3), box = 128 bytes x 128 rows,
+// 128-byte swizzle; rows past the end read as zero.
+static inline bool make_tmap_u8(CUtensorMap* tm, const void* ptr, int row_bytes, int64_t rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cuuint64_t(row_bytes), cuuint64_t(rows)};
+    cuuint64_t strides[1] = {cuuint64_t(row_bytes)};
+    cuuint32_t box[2] = {128, 128};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace moc

@@ -313,6 +313,41 @@ moc_status moc_attention_fwd_static(const moc_layout* layout, int B, int H, int 
  * after the call whose errors matter and before the next one. */
 moc_status moc_check_device_error_static(int32_t* detail, moc_stream_t stream);
 
+/* E4M3 variant of the attention stage (the pages' future-work lists: "Mixture
+ * of Contexts for Long Video Generation | Summary", limitations, and the
+ * jxzklqfsx.com write-up, "局限性與未來工作", name quantisation).
+ *
+ * moc_quantize_e4m3: per (b, h) slice of X (device bf16 [BH][L][d]) a scale
+ * that is a power of two, scale = 2^ceil(log2(amax / 448)) (1 for an all-zero
+ * slice), written to scale[BH] (device fp32), and X8 = E4M3(X / scale)
+ * (device bytes [BH][L][d], OCP E4M3 as in NVIDIA's e4m3 type, round to
+ * nearest even; X / scale is exact and never exceeds 448). X8 * scale is then
+ * exactly representable in bf16. */
+moc_status moc_quantize_e4m3(int BH, int64_t L, int d, const void* X, void* X8, float* scale,
+                             moc_stream_t stream);
+
+/* (4) on E4M3 inputs from moc_quantize_e4m3 (d = 128 only; other d return
+ * MOC_ERR_UNSUPPORTED): S = Q8 K8^T and O += P V8 on kind::f8f6f4 tensor cores,
+ * scores scaled by q_scale[bh] k_scale[bh] softmax_scale, P = exp of the scaled
+ * scores minus the running max, written to TMEM as E4M3 of P * 2^6 (the running
+ * max is raised once it grows by more than 2^2, so P * 2^6 <= 256 < 448), the
+ * row sum taken in fp32 on the unrounded P, O scaled by v_scale[bh] at the end.
+ * Writes the same partial rows and log-sum-exps as (4), for (5). Needs the
+ * workspace filled by (3). */
+moc_status moc_attend_partials_e4m3(const moc_layout* layout, int B, int H, int d, const void* Q8,
+                                    const void* K8, const void* V8, const float* q_scale,
+                                    const float* k_scale, const float* v_scale, int k,
+                                    float softmax_scale, void* ws, size_t ws_bytes,
+                                    moc_stream_t stream);
+
+/* (3), moc_attend_partials_e4m3 and (5) in order on one stream: the attention
+ * stage on E4M3 inputs, bf16 O and fp32 lse out as moc_attention_fwd. */
+moc_status moc_attention_fwd_e4m3(const moc_layout* layout, int B, int H, int d, const void* Q8,
+                                  const void* K8, const void* V8, const float* q_scale,
+                                  const float* k_scale, const float* v_scale, const int32_t* sel,
+                                  int k, float softmax_scale, void* O, float* lse, void* ws,
+                                  size_t ws_bytes, moc_stream_t stream);
+
 /* Whole forward pass on HOST buffers: (1) pooling, (2) routing (when k > 0)
  * and (3)-(5) for every (b, h) slice, the end-to-end call for inputs that live
  * in host memory. Q, K, V: host bf16 [B][H][L][d] (page-locked memory lets the

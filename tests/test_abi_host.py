@@ -17,7 +17,7 @@ from conftest import ROOT
 def _declared_functions():
     src = open(os.path.join(ROOT, "include", "moc.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    names = re.findall(r"\b(moc_[a-z_]+)\s*\(", src)
+    names = re.findall(r"\b(moc_[a-z0-9_]+)\s*\(", src)
     return sorted(set(names))
 
 
