@@ -394,6 +394,8 @@ def run_ours(args):
         line["gather"] = gather
     if not args.no_backward:
         line["backward"] = backward_timing(moc, lay, Q, K, V, O, lse, sel, k, pairs, d, stream)
+    if d == 128 and not args.no_e4m3:
+        line["e4m3_variant"] = e4m3_timing(moc, lay, Q, K, V, O, sel, k, ws, scale, stream, pairs, peak_tf)
     if ws_ == 1 and not args.no_dense_compare and wl.name == "eight":
         line["dense_compare"] = dense_compare(moc, wl, Q, K, V, O, lse, stream, pairs,
                                               stage_ms, ms_per_step, peak_tf)
@@ -480,6 +482,47 @@ def fused_timing(moc, lay, Q, K, V, sel, k, ws, scale, stream, B, H, L, reps=3):
     moc.check_device_error(ws)
     del O2, lse2
     return {"attend_merged_ms": statistics.mean(ts)}
+
+
+def e4m3_timing(moc, lay, Q, K, V, O_ref, sel, k, ws, scale, stream, pairs, peak_tf, reps=3):
+    """The E4M3 variant of the attention stage on the step's inputs and
+    selection: per-slice quantisation of Q, K, V (moc_quantize_e4m3), then
+    query lists, the E4M3 attention and the merge (moc_attention_fwd_e4m3);
+    CUDA events, mean of ``reps`` after one untimed run. Its output is compared
+    with the bf16 path's O of the same step (the effect of E4M3 inputs)."""
+    B, H, L, d = Q.shape
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record(stream)
+    (Q8, qs), (K8, ks), (V8, vs) = (moc.quantize_e4m3(t) for t in (Q, K, V))
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    quant_ms = ev[0].elapsed_time(ev[1])
+    O8 = torch.empty_like(Q)
+    lse8 = torch.empty(B, H, L, dtype=torch.float32, device=Q.device)
+    att, tot = [], []
+    for it in range(1 + reps):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        e[0].record(stream)
+        moc.build_qlists(lay, sel, B, H, k, ws)
+        e[1].record(stream)
+        moc.lib().moc_attend_partials_e4m3(lay.handle, B, H, d, moc._ptr(Q8), moc._ptr(K8), moc._ptr(V8),
+                                           moc._ptr(qs), moc._ptr(ks), moc._ptr(vs), k, float(scale),
+                                           moc._ptr(ws), ws.numel(), moc._stream())
+        e[2].record(stream)
+        moc.merge(lay, sel, k, ws, O8, lse8)
+        e[3].record(stream)
+        torch.cuda.synchronize()
+        if it >= 1:
+            att.append(e[1].elapsed_time(e[2]))
+            tot.append(e[0].elapsed_time(e[3]))
+    moc.check_device_error(ws)
+    diff = (O8.float() - O_ref.float()).abs()
+    a_ms = statistics.mean(att)
+    out = {"quantize_ms": quant_ms, "attend_ms": a_ms, "attention_stage_ms": statistics.mean(tot),
+           "tflops_selected_pairs": 4.0 * d * pairs / (a_ms / 1e3) / 1e12,
+           "o_vs_bf16_path": {"max_abs": diff.max().item(), "mean_abs": diff.mean().item()}}
+    del Q8, K8, V8, O8, lse8
+    return out
 
 
 def backward_timing(moc, lay, Q, K, V, O, lse, sel, k, pairs, d, stream, reps=5):
@@ -673,6 +716,8 @@ def main():
     ap.add_argument("--heads", type=int, default=None,
                     help="run the scene with this many heads instead (small profiling captures)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-e4m3", action="store_true",
+                    help="skip the timing of the E4M3 variant of the attention stage")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the timing of the backward pass (moc_attention_bwd) after the forward steps")
     ap.add_argument("--shard", default="heads", choices=["heads", "replicas"],
