@@ -78,6 +78,7 @@ SIGNATURES = {
     "moc_layout_device_error": (_I, [_P, _P, _P]),
     "moc_selftest_bounded_wait": (_I, [_P, _P]),
     "moc_set_attend_schedule": (_I, [_I, _I]),
+    "moc_set_attend_kernel": (_I, [_I]),
     "moc_forward_host": (_I, [_P, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _P, _P, _P, _SZ, _I, _P]),
     "moc_forward_host_device_bytes": (_SZ, [_P, _I, _I, _I, _I, _I]),
     "moc_route_perturb": (_I, [_P, _I, _I, _I, _I, _P, _P, _F, _F, _I, _P, _P]),
@@ -405,6 +406,12 @@ def check_layout_error(layout: Layout) -> int:
     _check(lib().moc_layout_device_error(layout.handle, ctypes.byref(det), _stream()),
            "layout device error word")
     return det.value
+
+
+def set_attend_kernel(variant: int = 0):
+    """Kernel of the attention stage for the following calls
+    (moc_set_attend_kernel): 0 default, 1 single CTA, 2 CTA pairs."""
+    _check(lib().moc_set_attend_kernel(int(variant)), "moc_set_attend_kernel")
 
 
 def set_attend_schedule(n_ctas: int = 0, reverse: bool = False):

@@ -34,11 +34,15 @@ moc_status check_common(const moc_layout* lay, int B, int H, int d, int k) {
 
 namespace {
 
-std::atomic<int> g_sched_ctas{0}, g_sched_reverse{0};
+std::atomic<int> g_sched_ctas{0}, g_sched_reverse{0}, g_attend_kernel{0};
+// the attention stage runs on CTA pairs where that kernel exists (d = 128)
+constexpr bool kPairByDefault = false;
 
 }  // namespace
 
 namespace moc {
+
+int attend_kernel_choice() { return g_attend_kernel.load(std::memory_order_relaxed); }
 
 AttendSchedule attend_schedule() {
     AttendSchedule s;
@@ -61,6 +65,7 @@ WsPlan plan_workspace(const moc_layout* lay, int B, int H, int d, int k) {
     p.blk_count = take(BH * size_t(p.nblk) * C * sizeof(int32_t));
     p.qoff = take((BH * C + 1) * sizeof(int32_t));
     p.tile_off = take((BH * C + 1) * sizeof(int32_t));
+    p.tile2_off = take((BH * C + 1) * sizeof(int32_t));
     p.qlist = take(BH * L * size_t(k) * sizeof(int32_t));
     p.lse_p = take(BH * L * S * sizeof(float));
     p.o_p = take(BH * L * S * size_t(d) * sizeof(float));
@@ -219,6 +224,12 @@ extern "C" moc_status moc_attend_partials(const moc_layout* lay, int B, int H, i
     if ((st = check_ws(lay, B, H, d, k, ws, ws_bytes, &p)) != MOC_OK) return st;
     if (!Q || !K || !V || !aligned16(Q) || !aligned16(K) || !aligned16(V)) return MOC_ERR_INVALID_ARG;
     if (!(scale > 0.0f) || scale != scale) return MOC_ERR_INVALID_ARG;
+    const int variant = moc::attend_kernel_choice();
+    if (variant == 2 && !moc::attend_pair_supported(d)) return MOC_ERR_INVALID_ARG;
+    if (variant == 2 || (variant == 0 && kPairByDefault && moc::attend_pair_supported(d)))
+        return cuda_status(moc::launch_attend_pair(lay->dv, B * H, d, Q, K, V, k, scale,
+                                                   int64_t(B) * H * lay->total_atiles2, static_cast<char*>(ws), p,
+                                                   (cudaStream_t)stream));
     const int64_t n_anchor = int64_t(B) * H * lay->total_atiles;
     return cuda_status(moc::launch_attend_tc(lay->dv, B * H, d, Q, K, V, k, scale, n_anchor,
                                              static_cast<char*>(ws), p, (cudaStream_t)stream));
@@ -290,6 +301,12 @@ extern "C" moc_status moc_check_device_error(void* ws, size_t ws_bytes, int32_t*
     }
     if (h[0] == moc::ERR_TIMEOUT) return MOC_ERR_DEVICE_TIMEOUT;
     if (h[0] == moc::ERR_CHECK) return MOC_ERR_DEVICE_CHECK;
+    return MOC_OK;
+}
+
+extern "C" moc_status moc_set_attend_kernel(int variant) {
+    if (variant < 0 || variant > 2) return MOC_ERR_INVALID_ARG;
+    g_attend_kernel.store(variant, std::memory_order_relaxed);
     return MOC_OK;
 }
 

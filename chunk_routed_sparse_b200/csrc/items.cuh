@@ -25,17 +25,20 @@ struct Item {
     int r_beg, r_end, k0, k1;
 };
 
-__device__ __forceinline__ bool decode(const DevLayout& dv, int BH, int64_t n_anchor, int64_t item,
-                                       const int32_t* tile_off, const int32_t* qoff,
-                                       const int32_t* qlist, Item& it) {
+// Item `item` of ROWS-row items: atab is the prefix of anchor items per group (in
+// a_order), tile_off the prefix of routed items per (b, h, chunk) list.
+template <int ROWS>
+__device__ __forceinline__ bool decode_rows(const DevLayout& dv, const int32_t* atab, int BH, int64_t n_anchor,
+                                            int64_t item, const int32_t* tile_off, const int32_t* qoff,
+                                            const int32_t* qlist, Item& it) {
     if (item < n_anchor) {
-        const int pos = upper_index(dv.atile_off, dv.G + 1, item / BH);
-        const int64_t local = item - int64_t(BH) * dv.atile_off[pos];
-        const int nt = dv.atile_off[pos + 1] - dv.atile_off[pos];
+        const int pos = upper_index(atab, dv.G + 1, item / BH);
+        const int64_t local = item - int64_t(BH) * atab[pos];
+        const int nt = atab[pos + 1] - atab[pos];
         const int g = dv.a_order[pos];
         it.bh = int(local / nt);
-        it.q0 = dv.grp_q0[g] + int(local % nt) * kItemRows;
-        it.nq = min(kItemRows, dv.grp_q1[g] - it.q0);
+        it.q0 = dv.grp_q0[g] + int(local % nt) * ROWS;
+        it.nq = min(ROWS, dv.grp_q1[g] - it.q0);
         it.slot_fixed = 0;
         it.entries = nullptr;
         it.r_beg = dv.ar_off[g];
@@ -49,8 +52,8 @@ __device__ __forceinline__ bool decode(const DevLayout& dv, int BH, int64_t n_an
     const int x = upper_index(tile_off, int(nlists + 1), r);
     const int c = x % dv.C;
     it.bh = x / dv.C;
-    const int e0 = qoff[x] + int(r - tile_off[x]) * kItemRows;
-    it.nq = min(kItemRows, qoff[x + 1] - e0);
+    const int e0 = qoff[x] + int(r - tile_off[x]) * ROWS;
+    it.nq = min(ROWS, qoff[x + 1] - e0);
     it.entries = qlist + e0;
     it.slot_fixed = -1;
     it.q0 = 0;
@@ -58,6 +61,13 @@ __device__ __forceinline__ bool decode(const DevLayout& dv, int BH, int64_t n_an
     it.k0 = dv.chunk_off[c];
     it.k1 = dv.chunk_off[c + 1];
     return true;
+}
+
+// Items of kItemRows rows (the layout's atile_off, the workspace's tile_off).
+__device__ __forceinline__ bool decode(const DevLayout& dv, int BH, int64_t n_anchor, int64_t item,
+                                       const int32_t* tile_off, const int32_t* qoff, const int32_t* qlist,
+                                       Item& it) {
+    return decode_rows<kItemRows>(dv, dv.atile_off, BH, n_anchor, item, tile_off, qoff, qlist, it);
 }
 
 // Key tiles of an item, in order: each range cut into 128-key tiles.

@@ -74,12 +74,17 @@ struct Cfg {
     static constexpr int kSlabs = D * kEB / 128;            // 128-byte slabs per row
     static constexpr int kSlabBytes = 128 * 128;            // 128 rows x 128 B
     static constexpr int kTileBytes = kSlabs * kSlabBytes;  // a 128-row Q, K or V tile
+    // K / V ring depths (a third stage of either, the one more tile that fits at
+    // d = 128, measured no faster: the copies are not latency-bound)
+    static constexpr int kKSt = 2;
+    static constexpr int kVSt = 2;
     static constexpr int oQ = 0;                            // Q_A, Q_B
-    static constexpr int oK = oQ + 2 * kTileBytes;          // 2 stages
-    static constexpr int oV = oK + 2 * kTileBytes;          // 2 stages
-    static constexpr int oBar = oV + 2 * kTileBytes;
+    static constexpr int oK = oQ + 2 * kTileBytes;          // kKSt stages
+    static constexpr int oV = oK + kKSt * kTileBytes;       // kVSt stages
+    static constexpr int oBar = oV + kVSt * kTileBytes;
     // + 1024 B alignment slack; at least 120 KB so that one CTA owns an SM (and its TMEM)
-    static constexpr int kSmem = (oBar + 256 + 1024) > 120 * 1024 ? (oBar + 256 + 1024) : 120 * 1024;
+    static constexpr int kSmem = (oBar + 512 + 1024) > 120 * 1024 ? (oBar + 512 + 1024) : 120 * 1024;
+    static_assert(kSmem <= 232448, "shared memory per CTA");
     static constexpr uint32_t kIdescQK = F8 ? idesc_e4m3_f32(128, kKT, 0) : idesc_bf16_f32(128, kKT, 0);
     static constexpr uint32_t kIdescPV = F8 ? idesc_e4m3_f32(128, D, 1) : idesc_bf16_f32(128, D, 1);
     // E4M3 P carries a factor 2^6 (and O is rescaled once the row max grows by more
@@ -95,12 +100,11 @@ __device__ __forceinline__ uint32_t col_o(int q) { return q ? 384u : 256u; }
 
 // mbarrier slots (8 bytes each) from Cfg::oBar; [x] = tile A / B or ring slot
 enum {
-    B_ITEM_FULL = 0, B_ITEM_EMPTY = 2, B_K_FULL = 4, B_K_EMPTY = 6, B_Q_FULL = 8,
-    B_S_FULL = 10, B_P_FULL = 12, B_PV_DONE = 14, B_V_FULL = 16, B_V_EMPTY = 18,
-    B_MMA_DONE = 20, B_COUNT = 21
+    B_ITEM_FULL = 0, B_ITEM_EMPTY = 2, B_Q_FULL = 4, B_S_FULL = 6, B_P_FULL = 8, B_PV_DONE = 10,
+    B_MMA_DONE = 12, B_K_FULL = 13, B_K_EMPTY = 16, B_V_FULL = 19, B_V_EMPTY = 22, B_COUNT = 25
 };
 
-struct Shared {  // at oBar + 192
+struct Shared {  // at oBar + 256
     int item[2];
     uint32_t tmem_base;
     int abort;
@@ -131,7 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     unsigned char* gbase = smem_raw + (base - raw);
     const uint32_t sQ = base + C::oQ, sK = base + C::oK, sV = base + C::oV;
     const uint32_t sBar = base + C::oBar;
-    Shared& sh = *reinterpret_cast<Shared*>(gbase + C::oBar + 192);
+    Shared& sh = *reinterpret_cast<Shared*>(gbase + C::oBar + 256);
     volatile int* abort = &sh.abort;
     auto bar = [&](int i) { return sBar + 8u * uint32_t(i); };
 
@@ -143,14 +147,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int x = 0; x < 2; ++x) {
             mbar_init(bar(B_ITEM_FULL + x), 1);
             mbar_init(bar(B_ITEM_EMPTY + x), 1 + 256);
-            mbar_init(bar(B_K_FULL + x), 1);
-            mbar_init(bar(B_K_EMPTY + x), 1);
-            mbar_init(bar(B_V_FULL + x), 1);
-            mbar_init(bar(B_V_EMPTY + x), 1);
             mbar_init(bar(B_Q_FULL + x), 128);
             mbar_init(bar(B_S_FULL + x), 1);
             mbar_init(bar(B_P_FULL + x), 128);
             mbar_init(bar(B_PV_DONE + x), 1);
+        }
+        for (int x = 0; x < C::kKSt; ++x) {
+            mbar_init(bar(B_K_FULL + x), 1);
+            mbar_init(bar(B_K_EMPTY + x), 1);
+        }
+        for (int x = 0; x < C::kVSt; ++x) {
+            mbar_init(bar(B_V_FULL + x), 1);
+            mbar_init(bar(B_V_EMPTY + x), 1);
         }
         mbar_init(bar(B_MMA_DONE), 1);
         sh.abort = 0;
@@ -199,18 +207,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     cur.next(key0, nvalid);
                     // K and V have rings of their own: K(j) is released once S(j) is computed,
                     // long before V(j) is released by PV(j), so K(j+2) streams in early
-                    const int st = gt & 1;
-                    const uint32_t par = ((gt >> 1) & 1) ^ 1;
-                    if (!wait_bar(bar(B_K_EMPTY + st), par, abort, hdr, 2)) { stop = true; break; }
+                    const int st = gt % C::kKSt, sv = gt % C::kVSt;
+                    if (!wait_bar(bar(B_K_EMPTY + st), ((gt / C::kKSt) & 1) ^ 1, abort, hdr, 2)) { stop = true; break; }
                     mbar_expect_tx(bar(B_K_FULL + st), C::kTileBytes);
 #pragma unroll
                     for (int s = 0; s < C::kSlabs; ++s)
                         tma_load_2d(sK + st * C::kTileBytes + s * C::kSlabBytes, &tmK, bar(B_K_FULL + st), 64 * s, row0 + key0);
-                    if (!wait_bar(bar(B_V_EMPTY + st), par, abort, hdr, 8)) { stop = true; break; }
-                    mbar_expect_tx(bar(B_V_FULL + st), C::kTileBytes);
+                    if (!wait_bar(bar(B_V_EMPTY + sv), ((gt / C::kVSt) & 1) ^ 1, abort, hdr, 8)) { stop = true; break; }
+                    mbar_expect_tx(bar(B_V_FULL + sv), C::kTileBytes);
 #pragma unroll
                     for (int s = 0; s < C::kSlabs; ++s)
-                        tma_load_2d(sV + st * C::kTileBytes + s * C::kSlabBytes, &tmV, bar(B_V_FULL + st), 64 * s, row0 + key0);
+                        tma_load_2d(sV + sv * C::kTileBytes + s * C::kSlabBytes, &tmV, bar(B_V_FULL + sv), 64 * s, row0 + key0);
                     ++gt;
                 }
                 if (stop) break;
@@ -218,11 +225,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             // drain: the last use of each stage has landed before the CTA exits (a load
             // cut short by an abort may have issued K without V; its V wait then times out
             // harmlessly because nothing was issued on it)
-            for (uint32_t g = (gt >= 2 ? gt - 2 : 0); g < gt; ++g) {
-                const uint32_t st = g & 1, par = (g >> 1) & 1;
-                for (int b = 0; b < 2; ++b) {
+            for (int b = 0; b < 2; ++b) {
+                const uint32_t n = b ? C::kVSt : C::kKSt;
+                for (uint32_t g = (gt >= n ? gt - n : 0); g < gt; ++g) {
                     const uint64_t t0 = globaltimer();
-                    while (!mbar_try_wait(bar((b ? B_V_FULL : B_K_FULL) + st), par)) {
+                    while (!mbar_try_wait(bar((b ? B_V_FULL : B_K_FULL) + g % n), (g / n) & 1)) {
                         if (globaltimer() - t0 > kTimeoutNs) { set_error(hdr, ERR_TIMEOUT, 9); break; }
                     }
                 }
@@ -251,13 +258,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (stop) break;
                 tc_fence_after();
                 for (int j = 0; j <= T && !stop; ++j) {
-                    const uint32_t st = gt & 1;
+                    const uint32_t st = gt % C::kKSt;
                     bool k_ready = false, v_ready = false;
                     for (int q = 0; q < nt; ++q) {
                         if (j > 0) {  // O_q += P_q(j-1) V(j-1)
-                            const uint32_t g = gtt[q] - 1, pst = (gt - 1) & 1;
+                            const uint32_t g = gtt[q] - 1, pst = (gt - 1) % C::kVSt;
                             if (!v_ready) {
-                                if (!wait_bar(bar(B_V_FULL + pst), ((gt - 1) >> 1) & 1, abort, hdr, 15)) { stop = true; break; }
+                                if (!wait_bar(bar(B_V_FULL + pst), ((gt - 1) / C::kVSt) & 1, abort, hdr, 15)) { stop = true; break; }
                                 v_ready = true;
                             }
                             if (!wait_bar(bar(B_P_FULL + q), g & 1, abort, hdr, 7)) { stop = true; break; }
@@ -276,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         if (j < T) {  // S_q(j) = Q_q K(j)^T, after PV_q(j-1) has read P_q(j-1)
                             if (!k_ready) {
-                                if (!wait_bar(bar(B_K_FULL + st), (gt >> 1) & 1, abort, hdr, 5)) { stop = true; break; }
+                                if (!wait_bar(bar(B_K_FULL + st), (gt / C::kKSt) & 1, abort, hdr, 5)) { stop = true; break; }
                                 k_ready = true;
                                 tc_fence_after();
                             }
@@ -297,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                     if (stop) break;
-                    if (j > 0) umma_commit(bar(B_V_EMPTY + ((gt - 1) & 1)));  // V(j-1) read by PV
+                    if (j > 0) umma_commit(bar(B_V_EMPTY + (gt - 1) % C::kVSt));  // V(j-1) read by PV
                     if (j < T) umma_commit(bar(B_K_EMPTY + st));              // K(j) read by S
                     if (j < T) ++gt;
                 }

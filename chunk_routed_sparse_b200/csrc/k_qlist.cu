@@ -38,11 +38,12 @@ __global__ void __launch_bounds__(32) qlist_count(int L, int C, int k, int nblk,
 
 // Per (bh): blk_count -> exclusive offsets of each block within each chunk's
 // list (in place); qoff[bh*C + c] <- list length, tile_off[bh*C + c] <- attention
-// work items of kItemRows entries.
+// work items of kItemRows entries, tile2_off[bh*C + c] <- items of kPairRows entries.
 __global__ void __launch_bounds__(256) qlist_scan_blocks(int C, int nblk,
                                                          int32_t* __restrict__ blk_count,
                                                          int32_t* __restrict__ qlen,
-                                                         int32_t* __restrict__ ntile) {
+                                                         int32_t* __restrict__ ntile,
+                                                         int32_t* __restrict__ ntile2) {
     const int bh = blockIdx.x;
     for (int c = threadIdx.x; c < C; c += blockDim.x) {
         int32_t run = 0;
@@ -54,48 +55,69 @@ __global__ void __launch_bounds__(256) qlist_scan_blocks(int C, int nblk,
         }
         qlen[size_t(bh) * C + c] = run;
         ntile[size_t(bh) * C + c] = (run + kItemRows - 1) / kItemRows;
+        ntile2[size_t(bh) * C + c] = (run + kPairRows - 1) / kPairRows;
     }
 }
 
-// In-place exclusive scan of two int32 arrays of n values (+ total at [n]),
+// In-place exclusive scan of three int32 arrays of n values (+ total at [n]),
 // one CTA of 1024 threads.
-__global__ void __launch_bounds__(1024) qlist_scan_global(int64_t n, int32_t* __restrict__ a,
-                                                          int32_t* __restrict__ b) {
-    __shared__ int32_t wa[32], wb[32];
-    __shared__ int32_t carry_a, carry_b;
+__global__ void __launch_bounds__(1024) qlist_scan_global(int64_t n, int32_t* __restrict__ a0,
+                                                          int32_t* __restrict__ a1, int32_t* __restrict__ a2) {
+    constexpr int NA = 3;
+    int32_t* const arr[NA] = {a0, a1, a2};
+    __shared__ int32_t w[NA][32];
+    __shared__ int32_t carry[NA];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (tid == 0) carry_a = carry_b = 0;
+    if (tid < NA) carry[tid] = 0;
     __syncthreads();
     for (int64_t base = 0; base < n; base += 1024) {
         const int64_t i = base + tid;
-        const int32_t va = (i < n) ? a[i] : 0, vb = (i < n) ? b[i] : 0;
-        int32_t xa = va, xb = vb;
+        int32_t v[NA], x[NA];
+#pragma unroll
+        for (int j = 0; j < NA; ++j) x[j] = v[j] = (i < n) ? arr[j][i] : 0;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const int32_t ya = __shfl_up_sync(0xffffffffu, xa, o), yb = __shfl_up_sync(0xffffffffu, xb, o);
-            if (lane >= o) { xa += ya; xb += yb; }
+#pragma unroll
+            for (int j = 0; j < NA; ++j) {
+                const int32_t y = __shfl_up_sync(0xffffffffu, x[j], o);
+                if (lane >= o) x[j] += y;
+            }
         }
-        if (lane == 31) { wa[warp] = xa; wb[warp] = xb; }
+        if (lane == 31) {
+#pragma unroll
+            for (int j = 0; j < NA; ++j) w[j][warp] = x[j];
+        }
         __syncthreads();
         if (warp == 0) {
-            int32_t sa = wa[lane], sb = wb[lane];
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int32_t ya = __shfl_up_sync(0xffffffffu, sa, o), yb = __shfl_up_sync(0xffffffffu, sb, o);
-                if (lane >= o) { sa += ya; sb += yb; }
+            for (int j = 0; j < NA; ++j) {
+                int32_t sj = w[j][lane];
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int32_t y = __shfl_up_sync(0xffffffffu, sj, o);
+                    if (lane >= o) sj += y;
+                }
+                w[j][lane] = sj;
             }
-            wa[lane] = sa;
-            wb[lane] = sb;
         }
         __syncthreads();
-        const int32_t pa = carry_a + (warp ? wa[warp - 1] : 0) + xa - va;
-        const int32_t pb = carry_b + (warp ? wb[warp - 1] : 0) + xb - vb;
-        if (i < n) { a[i] = pa; b[i] = pb; }
+        int32_t pre[NA];
+#pragma unroll
+        for (int j = 0; j < NA; ++j) {
+            pre[j] = carry[j] + (warp ? w[j][warp - 1] : 0) + x[j] - v[j];
+            if (i < n) arr[j][i] = pre[j];
+        }
         __syncthreads();
-        if (tid == 1023) { carry_a = pa + va; carry_b = pb + vb; }
+        if (tid == 1023) {
+#pragma unroll
+            for (int j = 0; j < NA; ++j) carry[j] = pre[j] + v[j];
+        }
         __syncthreads();
     }
-    if (tid == 0) { a[n] = carry_a; b[n] = carry_b; }
+    if (tid == 0) {
+#pragma unroll
+        for (int j = 0; j < NA; ++j) arr[j][n] = carry[j];
+    }
 }
 
 __global__ void __launch_bounds__(32) qlist_scatter(int L, int C, int k, int nblk,
@@ -139,11 +161,13 @@ cudaError_t launch_qlists(const DevLayout& dv, int BH, int k, const int32_t* sel
     int32_t* blk_count = reinterpret_cast<int32_t*>(ws + p.blk_count);
     int32_t* qoff = reinterpret_cast<int32_t*>(ws + p.qoff);
     int32_t* tile_off = reinterpret_cast<int32_t*>(ws + p.tile_off);
+    int32_t* tile2_off = reinterpret_cast<int32_t*>(ws + p.tile2_off);
     int32_t* qlist = reinterpret_cast<int32_t*>(ws + p.qlist);
     const int64_t n = int64_t(BH) * dv.C;
     if (k == 0) {  // no routed work: empty lists
         e = cudaMemsetAsync(qoff, 0, size_t(n + 1) * sizeof(int32_t), s);
         if (e == cudaSuccess) e = cudaMemsetAsync(tile_off, 0, size_t(n + 1) * sizeof(int32_t), s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(tile2_off, 0, size_t(n + 1) * sizeof(int32_t), s);
         return e;
     }
     if (BH > 65535) return cudaErrorInvalidValue;
@@ -156,8 +180,8 @@ cudaError_t launch_qlists(const DevLayout& dv, int BH, int k, const int32_t* sel
     }
     dim3 grid(p.nblk, BH);
     qlist_count<<<grid, 32, smem, s>>>(dv.L, dv.C, k, p.nblk, sel, blk_count, hdr);
-    qlist_scan_blocks<<<BH, 256, 0, s>>>(dv.C, p.nblk, blk_count, qoff, tile_off);
-    qlist_scan_global<<<1, 1024, 0, s>>>(n, qoff, tile_off);
+    qlist_scan_blocks<<<BH, 256, 0, s>>>(dv.C, p.nblk, blk_count, qoff, tile_off, tile2_off);
+    qlist_scan_global<<<1, 1024, 0, s>>>(n, qoff, tile_off, tile2_off);
     qlist_scatter<<<grid, 32, smem, s>>>(dv.L, dv.C, k, p.nblk, sel, blk_count, qoff, qlist);
     return cudaGetLastError();
 }

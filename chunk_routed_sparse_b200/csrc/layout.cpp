@@ -203,6 +203,13 @@ moc_status build_host(const moc_layout_desc* d, moc_layout* lay) {
         lay->atile_off.push_back(lay->atile_off.back() + (nq + moc::kItemRows - 1) / moc::kItemRows);
     }
     lay->total_atiles = lay->atile_off.back();
+    lay->atile2_off.assign(1, 0);
+    for (int x = 0; x < G; ++x) {
+        const int g = lay->a_order[x];
+        const int32_t nq = lay->grp_q1[g] - lay->grp_q0[g];
+        lay->atile2_off.push_back(lay->atile2_off.back() + (nq + moc::kPairRows - 1) / moc::kPairRows);
+    }
+    lay->total_atiles2 = lay->atile2_off.back();
 
     // Key blocks of the backward pass. Every key is attended by the queries of the
     // groups whose anchor ranges hold it and, for a video chunk, by the queries that
@@ -262,7 +269,7 @@ moc_status upload(moc_layout* lay) {
         &lay->cand_off, &lay->cand, &lay->cand_ncausal, &lay->rtile_off, &lay->atile_off,
         &lay->a_order, &lay->cand_seg, &lay->grp_seg, &lay->seg_voff, &lay->vid,
         &lay->rcost_full, &lay->rcost_causal, &lay->kb_range, &lay->kb_chunk, &lay->kb_goff,
-        &lay->kb_grp, &lay->kb_order, &lay->kt_off};
+        &lay->kb_grp, &lay->kb_order, &lay->kt_off, &lay->atile2_off};
     std::vector<size_t> offs;
     size_t total = 0;
     for (auto* t : tabs) {
@@ -316,6 +323,7 @@ moc_status upload(moc_layout* lay) {
     dv.kb_order = at(22);
     dv.kt_off = at(23);
     dv.kb_lead = lay->kb_lead;
+    dv.atile2_off = at(24);
     dv.err = reinterpret_cast<int32_t*>(static_cast<char*>(lay->dev_block) + err_off);
     return MOC_OK;
 }

@@ -12,6 +12,7 @@ namespace moc {
 
 constexpr int kQTile = 128;       // query rows per router tile and per attention MMA tile
 constexpr int kItemRows = 256;    // query rows per attention work item (two 128-row tiles)
+constexpr int kPairRows = 512;    // query rows per work item of the CTA-pair attention kernel
 constexpr int kMaxK = 31;         // top-k limit: 1+k partial slots fit one warp
 constexpr int kMaxChunks = 16384; // chunk limit (query-list counters live in shared memory)
 constexpr int kQlistBlock = 1024; // queries per block of the query-list builder
@@ -31,6 +32,7 @@ struct DevLayout {
     const int32_t* rtile_off;    // [G+1] prefix of router tiles (kQTile queries) per group
     const int32_t* atile_off;    // [G+1] prefix of anchor items (kItemRows queries), groups in a_order
     const int32_t* a_order;      // [G] groups by descending anchor keys per tile
+    const int32_t* atile2_off;   // [G+1] prefix of anchor items of kPairRows queries, groups in a_order
     int32_t S;                   // segments (shots) in stream order
     const int32_t* cand_seg;     // segment of every entry of cand
     const int32_t* grp_seg;      // [G] segment of the group's queries (-1: caption group)
@@ -59,9 +61,10 @@ struct moc_layout {
     int32_t max_cand = 0;       // largest candidate list of any group
     int64_t total_rtiles = 0;   // router tiles per (b, h)
     int64_t total_atiles = 0;   // anchor tiles per (b, h)
+    int64_t total_atiles2 = 0;  // anchor items of kPairRows queries per (b, h)
     std::vector<int32_t> chunk_off, kind, shot, frame;
     std::vector<int32_t> grp_q0, grp_q1, grp_kind, ar_off, ar, cand_off, cand, cand_ncausal;
-    std::vector<int32_t> rtile_off, atile_off, a_order;
+    std::vector<int32_t> rtile_off, atile_off, a_order, atile2_off;
     std::vector<int32_t> cand_seg, grp_seg, seg_voff, vid;  // segments (shots) in stream order
     std::vector<int32_t> rcost_full, rcost_causal;          // router tile cost prefixes
     std::vector<int64_t> grp_keys;  // anchor keys of each group
@@ -80,6 +83,7 @@ struct WsPlan {
     size_t blk_count = 0;  // int32 [BH][nblk][C]
     size_t qoff = 0;       // int32 [BH*C + 1] global start of every list
     size_t tile_off = 0;   // int32 [BH*C + 1] prefix of routed items (kItemRows entries each)
+    size_t tile2_off = 0;  // int32 [BH*C + 1] prefix of routed items of kPairRows entries
     size_t qlist = 0;      // int32 [BH*L*k] entries (query << 5 | slot)
     size_t lse_p = 0;      // fp32 [BH][L][1+k]
     size_t o_p = 0;        // fp32 [BH][L][1+k][d]
@@ -113,6 +117,13 @@ cudaError_t launch_qlists(const DevLayout& dv, int BH, int k, const int32_t* sel
 cudaError_t launch_attend_tc(const DevLayout& dv, int BH, int d, const void* Q, const void* K,
                              const void* V, int k, float scale, int64_t n_anchor_items, char* ws,
                              const WsPlan& p, cudaStream_t s);
+// (4) on CTA pairs (cta_group::2; bf16, d = 128 only): items of kPairRows rows,
+// n_anchor2 = B*H x the layout's total_atiles2, routed items from the plan's tile2_off.
+bool attend_pair_supported(int d);
+cudaError_t launch_attend_pair(const DevLayout& dv, int BH, int d, const void* Q, const void* K, const void* V,
+                               int k, float scale, int64_t n_anchor2, char* ws, const WsPlan& p, cudaStream_t s);
+// Kernel of the attention stage (moc_set_attend_kernel): 0 default, 1 single CTA, 2 CTA pairs.
+int attend_kernel_choice();
 cudaError_t launch_attend_merged(const DevLayout& dv, int BH, int d, const void* Q, const void* K,
                                  const void* V, int k, float scale, int64_t n_anchor, char* ws,
                                  const WsPlan& p, const int32_t* sel, void* O, float* lse, cudaStream_t s);

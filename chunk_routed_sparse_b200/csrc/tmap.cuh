@@ -38,6 +38,19 @@ static inline bool make_tmap(CUtensorMap* tm, const void* ptr, int d, int64_t ro
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [rows][d] bf16 matrix, box = 64 columns x box_rows rows, 128-byte swizzle.
+static inline bool make_tmap_box(CUtensorMap* tm, const void* ptr, int d, int64_t rows, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(rows)};
+    cuuint64_t strides[1] = {cuuint64_t(d) * 2};
+    cuuint32_t box[2] = {64, cuuint32_t(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // [rows][row_bytes] one-byte elements (E4M3), box = 128 bytes x 128 rows,
 // 128-byte swizzle; rows past the end read as zero.
 static inline bool make_tmap_u8(CUtensorMap* tm, const void* ptr, int row_bytes, int64_t rows) {

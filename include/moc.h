@@ -399,6 +399,16 @@ moc_status moc_selftest_bounded_wait(int32_t* dev_word, moc_stream_t stream);
  * tests use this to show it. Not thread-safe against concurrent launches. */
 moc_status moc_set_attend_schedule(int n_ctas, int item_order);
 
+/* Diagnostic (the pages have no counterpart): which kernel computes the
+ * attention stage (4) in the calls that follow in this process - 0 the default,
+ * 1 the single-CTA kernel, 2 the CTA-pair kernel (clusters of two SMs sharing
+ * every MMA, tcgen05 cta_group::2; bf16 with d = 128 only: other shapes then
+ * return MOC_ERR_INVALID_ARG). Both compute the same partials (Summary §3.1);
+ * their summation orders differ only inside the MMAs. Returns
+ * MOC_ERR_INVALID_ARG for another variant. Not thread-safe against concurrent
+ * launches. */
+moc_status moc_set_attend_kernel(int variant);
+
 /* Read and clear the device error word kept with a layout, where kernels that
  * run without a workspace (the router, (2)) record a bounded wait that gave up.
  * Synchronises the stream. Returns MOC_OK, MOC_ERR_DEVICE_TIMEOUT or

@@ -222,10 +222,12 @@ def test_qlists_invert_selection():
     nblk = (L + 1023) // 1024
     off_qoff = a(256) + a(BH * nblk * C * 4)
     off_tile = off_qoff + a((BH * C + 1) * 4)
-    off_list = off_tile + a((BH * C + 1) * 4)
+    off_tile2 = off_tile + a((BH * C + 1) * 4)
+    off_list = off_tile2 + a((BH * C + 1) * 4)
     wsc = ws.cpu()
     qoff = wsc[off_qoff:off_qoff + (BH * C + 1) * 4].view(torch.int32).numpy()
     tile = wsc[off_tile:off_tile + (BH * C + 1) * 4].view(torch.int32).numpy()
+    tile2 = wsc[off_tile2:off_tile2 + (BH * C + 1) * 4].view(torch.int32).numpy()
     n_valid = int((sel >= 0).sum())
     qlist = wsc[off_list:off_list + n_valid * 4].view(torch.int32).numpy()
     s = sel.cpu().numpy().reshape(BH, L, k)
@@ -240,6 +242,7 @@ def test_qlists_invert_selection():
             want = np.nonzero((s[bh] == c).any(-1))[0]
             assert np.array_equal(q, want)
             assert tile[x + 1] - tile[x] == (len(ent) + 255) // 256
+            assert tile2[x + 1] - tile2[x] == (len(ent) + 511) // 512
 
 
 def test_deterministic_repeat():
