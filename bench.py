@@ -41,6 +41,9 @@ import moc_workloads as W  # noqa: E402
 
 METRIC = "MoC fwd tokens/s and selected-pair TFLOP/s (% bf16 peak) at 180k tokens"
 STAGES = ["pool", "route", "qlist", "attend", "merge"]
+# kernel of the attention stage (moc_set_attend_kernel): the library's default, the
+# single-CTA kernel, or the CTA-pair kernel (bf16, d = 128)
+ATTEND_KERNELS = {"default": 0, "single": 1, "pair": 2}
 LAUNCHES_PER_STEP = {"pool": 1, "route": 1, "qlist": 4, "attend": 1, "merge": 1}
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -220,6 +223,7 @@ def run_ours(args):
 
     ws_, rank, local = dist_env()
     torch.cuda.set_device(local)
+    moc.set_attend_kernel(ATTEND_KERNELS[args.attend_kernel])
     if ws_ > 1:
         import datetime
         import torch.distributed as dist
@@ -366,7 +370,8 @@ def run_ours(args):
         "config": {"workload": workload_string(wl, lay.C),
                    "tokens_per_step_per_gpu": tokens if shard != "heads" else wl.B * L * H / (wl.B * wl.H),
                    "l2": "inputs larger than L2 (3 x %.2f GB), no flush" % (Q.numel() * 2 / 1e9),
-                   "parallelism": parallelism},
+                   "parallelism": parallelism,
+                   "attend_kernel": args.attend_kernel},
         "selected_pair_tflops_attend": achieved_tf,
         "selected_pair_tflops_step": 4.0 * d * job_pairs / (ms_per_step / 1e3) / 1e12,
         "pct_bf16_peak_attend": 100.0 * achieved_tf / peak_tf,
@@ -726,6 +731,8 @@ def main():
     ap.add_argument("--gather", action="store_true",
                     help="with --shard heads: all-gather the output slices after the timed steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--attend-kernel", default="default", choices=sorted(ATTEND_KERNELS),
+                    help="kernel of the attention stage (the CTA-pair kernel is a measured alternative)")
     ap.add_argument("--no-dense-compare", action="store_true",
                     help="skip the dense and FLOP-matched block-diagonal runs of the attention kernel")
     args = ap.parse_args()

@@ -32,10 +32,13 @@
 //   warps 0-3 / 4-7: softmax of this CTA's rows of pair tile A / B, one thread a
 //          row, exactly as in the single-CTA kernel; their arrivals that the MMA
 //          warp waits on go to CTA 0 (one per warp).
-// Every wait is bounded (2 s; ERR_TIMEOUT with a site code in the header). The
-// pair leaves together: each producer first waits until every stage it filled
-// was released (its copies landed, the commits on its barriers arrived), CTA 0
-// waits for its last MMA, then a cluster barrier, then the TMEM is freed.
+// Waits on barriers fed by another CTA's plain stores (the item slots, the gathered
+// Q rows) acquire at cluster scope; those fed by tcgen05 commits, TMA completion or
+// the P hand-off acquire at CTA scope. Every wait is bounded (2 s; ERR_TIMEOUT with
+// a site code in the header). The pair leaves together: each producer first waits
+// until every stage it filled was released (its copies landed, the commits on its
+// barriers arrived), CTA 0 waits for its last MMA, then a cluster barrier, then the
+// TMEM is freed.
 #include "items.cuh"
 #include "pipeline.cuh"
 #include "tmap.cuh"
@@ -112,9 +115,9 @@ __device__ __forceinline__ bool wait_cl_warp(uint32_t bar, uint32_t parity, vola
     const bool ok = wait_cl(bar, parity, abort, hdr, where);
     return __all_sync(0xffffffffu, ok);
 }
-// ignores the abort flag: outstanding copies and commits must land first
-__device__ __forceinline__ void drain_cl(uint32_t bar, uint32_t parity, uint64_t deadline, int32_t* hdr, int where) {
-    while (!mbar_try_wait_cluster(bar, parity)) {
+// bounded by `deadline`, ignoring the abort flag: outstanding copies and commits land first
+__device__ __forceinline__ void drain_until(uint32_t bar, uint32_t parity, uint64_t deadline, int32_t* hdr, int where) {
+    while (!mbar_try_wait(bar, parity)) {
         if (globaltimer() > deadline) {
             set_error(hdr, ERR_TIMEOUT, where);
             return;
@@ -212,13 +215,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     int key0, nvalid;
                     cur.next(key0, nvalid);
                     const int st = gt % kKSt, sv = gt % kVSt;
-                    if (!wait_cl(bar(B_K_EMPTY + st), ((gt / kKSt) & 1) ^ 1, abort, hdr, 2)) { stop = true; break; }
+                    if (!wait_bar(bar(B_K_EMPTY + st), ((gt / kKSt) & 1) ^ 1, abort, hdr, 2)) { stop = true; break; }
                     if (lead) mbar_expect_tx(bar(B_K_FULL + st), 2 * kKHalf);
 #pragma unroll
                     for (int s = 0; s < 2; ++s)
                         tma_load_2d_pair(sK + st * kKHalf + s * kKSlab, &tmK, lead_bar(B_K_FULL + st), 64 * s,
                                          row0 + key0 + 64 * int(rank));
-                    if (!wait_cl(bar(B_V_EMPTY + sv), ((gt / kVSt) & 1) ^ 1, abort, hdr, 8)) { stop = true; break; }
+                    if (!wait_bar(bar(B_V_EMPTY + sv), ((gt / kVSt) & 1) ^ 1, abort, hdr, 8)) { stop = true; break; }
                     if (lead) mbar_expect_tx(bar(B_V_FULL + sv), 2 * kVHalf);
                     tma_load_2d_pair(sV + sv * kVHalf, &tmV, lead_bar(B_V_FULL + sv), 64 * int(rank), row0 + key0);
                     ++gt;
@@ -229,9 +232,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             // (so its copies have landed and the commits on its barriers arrived)
             const uint64_t deadline = globaltimer() + kTimeoutNs;
             for (uint32_t g = (gt >= uint32_t(kKSt) ? gt - kKSt : 0); g < gt; ++g)
-                drain_cl(bar(B_K_EMPTY + g % kKSt), (g / kKSt) & 1, deadline, hdr, 9);
+                drain_until(bar(B_K_EMPTY + g % kKSt), (g / kKSt) & 1, deadline, hdr, 9);
             for (uint32_t g = (gt >= uint32_t(kVSt) ? gt - kVSt : 0); g < gt; ++g)
-                drain_cl(bar(B_V_EMPTY + g % kVSt), (g / kVSt) & 1, deadline, hdr, 18);
+                drain_until(bar(B_V_EMPTY + g % kVSt), (g / kVSt) & 1, deadline, hdr, 18);
         } else if (warp == 9 && lead && lane == 0) {
             // ------------------------------------------------------------ MMA issuer (CTA 0)
             uint32_t gt = 0;
@@ -259,10 +262,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         if (j > 0) {  // O_q += P_q(j-1) V(j-1)
                             const uint32_t g = gtt[q] - 1, pst = (gt - 1) % kVSt;
                             if (!v_ready) {
-                                if (!wait_cl(bar(B_V_FULL + pst), ((gt - 1) / kVSt) & 1, abort, hdr, 15)) { stop = true; break; }
+                                if (!wait_bar(bar(B_V_FULL + pst), ((gt - 1) / kVSt) & 1, abort, hdr, 15)) { stop = true; break; }
                                 v_ready = true;
                             }
-                            if (!wait_cl(bar(B_P_FULL + q), g & 1, abort, hdr, 7)) { stop = true; break; }
+                            if (!wait_bar(bar(B_P_FULL + q), g & 1, abort, hdr, 7)) { stop = true; break; }
                             tc_fence_after();
 #pragma unroll
                             for (int kk = 0; kk < kKT / 16; ++kk) {
@@ -274,7 +277,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         }
                         if (j < T) {  // S_q(j) = Q_q K(j)^T
                             if (!k_ready) {
-                                if (!wait_cl(bar(B_K_FULL + st), (gt / kKSt) & 1, abort, hdr, 5)) { stop = true; break; }
+                                if (!wait_bar(bar(B_K_FULL + st), (gt / kKSt) & 1, abort, hdr, 5)) { stop = true; break; }
                                 k_ready = true;
                                 tc_fence_after();
                             }
@@ -299,7 +302,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
             umma_commit_pair(bar(B_MMA_DONE), 1);
             const uint64_t deadline = globaltimer() + kTimeoutNs;
-            drain_cl(bar(B_MMA_DONE), 0, deadline, hdr, 10);
+            drain_until(bar(B_MMA_DONE), 0, deadline, hdr, 10);
         }
         __syncwarp();
     } else {
@@ -316,7 +319,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (!wait_cl_warp(bar(B_ITEM_FULL + slot), (it >> 1) & 1, abort, hdr, 11)) break;
             const int item = *reinterpret_cast<volatile int*>(&sh.item[slot]);
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(lead_bar(B_ITEM_EMPTY + slot));
+            if (lane == 0) {  // CTA 1's reads of the slot are released at cluster scope
+                if (lead) mbar_arrive(bar(B_ITEM_EMPTY + slot));
+                else mbar_arrive_cluster(lead_bar(B_ITEM_EMPTY + slot));
+            }
             if (item < 0) break;
             Item itm;
             decode_rows<kPairRows>(dv, dv.atile2_off, BH, n_anchor, item, tile2_off, qoff, qlist, itm);
@@ -352,7 +358,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(lead_bar(B_Q_FULL + q));
+            if (lane == 0) {  // CTA 1's gathered rows are released at cluster scope
+                if (lead) mbar_arrive(bar(B_Q_FULL + q));
+                else mbar_arrive_cluster(lead_bar(B_Q_FULL + q));
+            }
 
             Cursor cur;
             cur.init(dv, itm);
@@ -361,7 +370,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int j = 0; cur.more(); ++j) {
                 int key0, nvalid;
                 cur.next(key0, nvalid);
-                if (!wait_cl_warp(bar(B_S_FULL + q), gtt & 1, abort, hdr, 12)) { stop = true; break; }
+                if (!wait_bar_warp(bar(B_S_FULL + q), gtt & 1, abort, hdr, 12)) { stop = true; break; }
                 tc_fence_after();
                 uint32_t s[kKT];
 #pragma unroll
@@ -392,7 +401,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     rescale = true;
                 }
                 if (__any_sync(0xffffffffu, rescale)) {
-                    if (!wait_cl_warp(bar(B_PV_DONE + q), (gtt - 1) & 1, abort, hdr, 13)) { stop = true; break; }
+                    if (!wait_bar_warp(bar(B_PV_DONE + q), (gtt - 1) & 1, abort, hdr, 13)) { stop = true; break; }
                     tc_fence_after();
 #pragma unroll
                     for (int c = 0; c < D / 32; ++c) {
@@ -428,14 +437,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(lead_bar(B_P_FULL + q));
+                // P lives in TMEM, ordered by the tcgen05 fences: CTA 1's arrival needs no
+                // cluster-scope release (that fence on every tile cost ~15 %)
+                if (lane == 0) {
+                    if (lead) mbar_arrive(bar(B_P_FULL + q));
+                    else mbar_arrive_cluster_relaxed(lead_bar(B_P_FULL + q));
+                }
                 ++gtt;
             }
             if (stop) break;
             // epilogue: O / l -> partial row and its log-sum-exp, staged per 32-column
             // chunk in the warp's own rows of its Q tile (read by this item's S MMAs
             // only, all complete once the last PV_DONE is seen)
-            if (!wait_cl_warp(bar(B_PV_DONE + q), (gtt - 1) & 1, abort, hdr, 14)) break;
+            if (!wait_bar_warp(bar(B_PV_DONE + q), (gtt - 1) & 1, abort, hdr, 14)) break;
             tc_fence_after();
             const float inv = 1.f / l;
             float* dst = (my_tok >= 0) ? o_p + ((size_t(itm.bh) * L + my_tok) * S + my_slot) * D : nullptr;

@@ -236,6 +236,11 @@ __device__ __forceinline__ uint32_t mapa(uint32_t a, uint32_t rank) {
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+// without release semantics (no cluster-scope fence): for hand-offs whose data is
+// ordered otherwise (TMEM writes, by the tcgen05 fences around the arrival)
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cl_addr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cl_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
 }
