@@ -401,7 +401,7 @@ def run_ours(args):
         line["backward"] = backward_timing(moc, lay, Q, K, V, O, lse, sel, k, pairs, d, stream)
     if d == 128 and not args.no_e4m3:
         line["e4m3_variant"] = e4m3_timing(moc, lay, Q, K, V, O, sel, k, ws, scale, stream, pairs, peak_tf)
-    if ws_ == 1 and not args.no_dense_compare and wl.name == "eight":
+    if ws_ == 1 and not args.no_dense_compare:
         line["dense_compare"] = dense_compare(moc, wl, Q, K, V, O, lse, stream, pairs,
                                               stage_ms, ms_per_step, peak_tf)
     if rank == 0 and ws_ == 1 and not args.no_cpu_baseline:
@@ -414,35 +414,51 @@ def run_ours(args):
         torch.distributed.destroy_process_group()
 
 
+def flop_matched_blocks(L: int, pairs_per_head: float):
+    """Equal video blocks of s tokens (n of them, plus one block of the r left over)
+    whose block-diagonal dense attention keeps as many (query, key) pairs per head as
+    the MoC scene: n s^2 + r^2 closest to pairs_per_head, with n s + r = L."""
+    s0 = max(1, int(pairs_per_head // L))
+    best = None
+    for s_ in range(max(1, s0 - 4000), min(L, s0 + 4000) + 1):
+        n, r = divmod(L, s_)
+        err = abs(n * s_ * s_ + r * r - pairs_per_head)
+        if best is None or err < best[0]:
+            best = (err, s_, n, r)
+    return best[1], best[2], best[3]
+
+
 def dense_compare(moc, wl, Q, K, V, O, lse, stream, moc_pairs, stage_ms, moc_step_ms, peak_tf):
     """The same attention kernel on two anchor-only layouts of the scene's length
     (k = 0, so no routing and one partial per row):
       dense - one caption segment and one shot holding every frame, so every
               query attends every key (L^2 pairs per head);
-      flop_matched - seven shots of 6 x 28,405 + 10,082 tokens, block-diagonal
-              dense attention with the MoC scene's kept-pair count (within 0.02 %),
-              which separates the pruning gain from the cost of routing, query
-              lists, gathered tiles and the merge.
+      flop_matched - equal video blocks (``flop_matched_blocks``), block-diagonal
+              dense attention with the MoC scene's kept-pair count per head (within
+              0.1 %), which separates the pruning gain from the cost of routing,
+              query lists, gathered tiles and the merge.
     Pool -> attention (query lists, attend, merge) is timed with CUDA events over
     3 runs after 2 warm-up runs, on the resident Q, K, V."""
     import moc_workloads as Wm
-    L, d, H = wl.L, wl.d, wl.H
+    B, L, d, H = wl.B, wl.L, wl.d, wl.H
     n_cap = sum(sg.length for sg in wl.segments if sg.kind == Wm.CAPTION)
+    n_fr, rest = divmod(L - n_cap, 1500)
+    blk, n_blk, r_blk = flop_matched_blocks(L, moc_pairs / (B * H))
     scenes = {
         "dense": [Wm.Segment(n_cap, Wm.CAPTION, -1, -1)]
-                 + [Wm.Segment(1500, Wm.VIDEO, 0, f) for f in range((L - n_cap) // 1500)],
-        "flop_matched": [Wm.Segment(28405, Wm.VIDEO, s_, 0) for s_ in range(6)]
-                        + [Wm.Segment(L - 6 * 28405, Wm.VIDEO, 6, 0)],
+                 + [Wm.Segment(1500 + (rest if f == n_fr - 1 else 0), Wm.VIDEO, 0, f) for f in range(n_fr)],
+        "flop_matched": [Wm.Segment(blk, Wm.VIDEO, s_, 0) for s_ in range(n_blk)]
+                        + ([Wm.Segment(r_blk, Wm.VIDEO, n_blk, 0)] if r_blk else []),
     }
     out = {}
     for name, segs in scenes.items():
         assert sum(sg.length for sg in segs) == L
-        w2 = Wm.custom(name, 1, H, d, segs, anchor="shot", causal=True, k=0)
+        w2 = Wm.custom(name, B, H, d, segs, anchor="shot", causal=True, k=0)
         lay = moc.Layout.from_workload(w2, device=Q.device.index)
-        ws = moc.workspace(lay, 1, H, d, 0, Q.device)
-        kbar = torch.empty(1, H, lay.C, d, dtype=torch.float32, device=Q.device)
+        ws = moc.workspace(lay, B, H, d, 0, Q.device)
+        kbar = torch.empty(B, H, lay.C, d, dtype=torch.float32, device=Q.device)
         # dense: every query sees every key; block-diagonal: every query its own block
-        pairs = H * L * L if name == "dense" else H * sum(sg.length ** 2 for sg in segs)
+        pairs = B * H * L * L if name == "dense" else B * H * sum(sg.length ** 2 for sg in segs)
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         att, tot = [], []
         for it in range(5):
@@ -462,6 +478,7 @@ def dense_compare(moc, wl, Q, K, V, O, lse, stream, moc_pairs, stage_ms, moc_ste
                      "frac_sustained": 4.0 * d * pairs / (a / 1e3) / 1e12 / peak_tf}
         del ws
     moc_attention_ms = stage_ms["qlist"] + stage_ms["attend"] + stage_ms["merge"]
+    out["flop_matched"]["blocks"] = {"tokens": blk, "count": n_blk, "rest": r_blk}
     out["moc_pairs"] = moc_pairs
     out["moc_step_speedup_vs_dense"] = out["dense"]["step_ms"] / moc_step_ms
     out["moc_attention_vs_flop_matched"] = moc_attention_ms / out["flop_matched"]["attention_ms"]

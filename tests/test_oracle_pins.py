@@ -270,13 +270,17 @@ def test_near_tie_rule():
 def test_dense_comparison_layouts():
     """The benchmark's dense and FLOP-matched block-diagonal layouts (k = 0):
     the oracle's kept-pair counts are L^2 and the block sum of squares, and the
-    block-diagonal one matches the eight-shot scene's MoC count within 0.02 %."""
+    block-diagonal one (``bench.flop_matched_blocks``) matches the eight-shot
+    scene's MoC count within 0.02 %."""
+    import bench
     wl = W.eight()
     L = wl.L
     n_cap = sum(s.length for s in wl.segments if s.kind == W.CAPTION)
+    n_fr, rest = divmod(L - n_cap, 1500)
     dense = [W.Segment(n_cap, W.CAPTION, -1, -1)] + \
-        [W.Segment(1500, W.VIDEO, 0, f) for f in range((L - n_cap) // 1500)]
-    blocks = [W.Segment(28405, W.VIDEO, s, 0) for s in range(6)] + [W.Segment(L - 6 * 28405, W.VIDEO, 6, 0)]
+        [W.Segment(1500 + (rest if f == n_fr - 1 else 0), W.VIDEO, 0, f) for f in range(n_fr)]
+    blk, n_blk, r_blk = bench.flop_matched_blocks(L, 4_943_332_144)
+    blocks = [W.Segment(blk, W.VIDEO, s, 0) for s in range(n_blk)] + ([W.Segment(r_blk, W.VIDEO, n_blk, 0)] if r_blk else [])
     for segs, want in ((dense, L * L), (blocks, sum(s.length ** 2 for s in blocks))):
         w2 = W.custom("cmp", 1, 1, 128, segs, "shot", 0, True, 0, 1, "none")
         assert w2.L == L
