@@ -335,6 +335,34 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
     return d;
 }
 
+// 2^x for two values on the FMA pipe (for a share of the softmax exponentials, so
+// that the MUFU does not set the pace). Range reduction: x = n + f with n = round(x),
+// taken from the low mantissa bits of x + 1.5 * 2^23, f in [-1/2, 1/2]; 2^f by a
+// degree-4 polynomial (least-squares fit of 2^f on [-1/2, 1/2] with relative
+// weighting, coefficients rounded to fp32; relative error below 3e-6 in fp32
+// Horner form); 2^n added to the exponent field. x is first raised to -126, where
+// the result is not a normal number but below 2^-126.
+__device__ __forceinline__ uint64_t ex2_fma2(float xa, float xb) {
+    constexpr float kShift = 12582912.f;           // 1.5 * 2^23
+    constexpr int kShiftBits = 0x4B400000;         // its bit pattern
+    constexpr float c0 = 9.999991655e-01f, c1 = 6.931219697e-01f, c2 = 2.402498126e-01f,
+                    c3 = 5.591703951e-02f, c4 = 9.560510516e-03f;
+    const uint64_t x = f2_pack(fmaxf(xa, -126.f), fmaxf(xb, -126.f));
+    const uint64_t t = f2_add(x, f2_pack(kShift, kShift));           // kShift + n
+    const uint64_t n = f2_add(t, f2_pack(-kShift, -kShift));         // n exactly
+    const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), x);           // x - n
+    uint64_t p = f2_fma(f2_pack(c4, c4), f, f2_pack(c3, c3));
+    p = f2_fma(p, f, f2_pack(c2, c2));
+    p = f2_fma(p, f, f2_pack(c1, c1));
+    p = f2_fma(p, f, f2_pack(c0, c0));
+    float pa, pb, ta, tb;
+    f2_unpack(p, pa, pb);
+    f2_unpack(t, ta, tb);
+    pa = __int_as_float(__float_as_int(pa) + ((__float_as_int(ta) - kShiftBits) << 23));
+    pb = __int_as_float(__float_as_int(pb) + ((__float_as_int(tb) - kShiftBits) << 23));
+    return f2_pack(pa, pb);
+}
+
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
