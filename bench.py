@@ -223,6 +223,8 @@ def run_ours(args):
 
     ws_, rank, local = dist_env()
     torch.cuda.set_device(local)
+    if args.attend_kernel == "pair" and W.CONFIGS[args.config]().d != 128:
+        raise SystemExit("--attend-kernel pair: the CTA-pair kernel is built for d = 128 only")
     moc.set_attend_kernel(ATTEND_KERNELS[args.attend_kernel])
     if ws_ > 1:
         import datetime
