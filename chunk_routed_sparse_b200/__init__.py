@@ -336,6 +336,48 @@ def forward(layout: Layout, Q, K, V, k: int, causal: bool = True, scale=None, ws
     return O, lse, sel, kbar
 
 
+class MoCAttention(torch.autograd.Function):
+    """The MoC attention as a torch.autograd.Function ("Mixture of Contexts for Long
+    Video Generation | Summary", appendix on training: a custom autograd function
+    carries the gradient of the attention over the selected keys and values).
+
+    forward: pool -> route -> attention (moc_pool_keys, moc_route,
+    moc_attention_fwd); backward: moc_attention_bwd for the upstream gradient of O.
+    The top-k selection is discrete, so it is a constant of the backward pass: Q, K
+    and V receive the gradient of the attention over each query's anchors and
+    selected chunks, and nothing flows through the pooled keys or the scores. Every
+    step runs in the library's kernels; this class only marshals arguments and
+    keeps (Q, K, V, O, lse, sel) for the backward call.
+
+    apply(layout, Q, K, V, k, causal=True, scale=None) -> O (bf16 [B, H, L, d]);
+    the selection of the last call is left in ``MoCAttention.last_sel``."""
+
+    last_sel: Optional[torch.Tensor] = None
+
+    @staticmethod
+    def forward(ctx, layout, Q, K, V, k, causal=True, scale=None):
+        Q, K, V = Q.contiguous(), K.contiguous(), V.contiguous()
+        O, lse, sel, _ = forward(layout, Q, K, V, k, causal, scale)
+        ctx.layout, ctx.k, ctx.scale = layout, k, scale
+        ctx.save_for_backward(Q, K, V, O, lse, sel)
+        MoCAttention.last_sel = sel
+        return O
+
+    @staticmethod
+    def backward(ctx, dO):
+        Q, K, V, O, lse, sel = ctx.saved_tensors
+        dQ, dK, dV = attention_bwd(ctx.layout, Q, K, V, O, lse, dO.contiguous().to(torch.bfloat16), sel,
+                                   ctx.k, scale=ctx.scale)
+        return None, dQ, dK, dV, None, None, None
+
+
+def moc_attention(layout: Layout, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, k: int,
+                  causal: bool = True, scale: Optional[float] = None) -> torch.Tensor:
+    """Differentiable MoC attention (MoCAttention.apply): bf16 O with gradients for
+    Q, K and V through the library's backward pass."""
+    return MoCAttention.apply(layout, Q, K, V, k, causal, scale)
+
+
 def quantize_e4m3(X: torch.Tensor):
     """Per-(b, h) power-of-two scale and E4M3 bytes of a bf16 [B, H, L, d] tensor
     (moc_quantize_e4m3). Returns (X8 uint8 [B, H, L, d], scale fp32 [B, H])."""
