@@ -84,6 +84,17 @@ def test_small_ragged_scene_every_row(k, anchor):
     _check(_ragsmall(k=k, anchor=anchor))
 
 
+def test_non_causal_scene_every_row():
+    """Routing over earlier and later chunks: longer query lists per chunk."""
+    wl = _ragsmall(k=4)
+    _check(wl.replace(causal=False))
+
+
+def test_odd_head_count_every_row():
+    """B x H = 10 slices: items and clusters that do not divide evenly."""
+    _check(_ragsmall(B=2, H=5, k=3))
+
+
 def test_single_shot_clip_sampled():
     _check(W.single(), n_random=512, seed=3)
 
