@@ -349,10 +349,7 @@ class MoCAttention(torch.autograd.Function):
     step runs in the library's kernels; this class only marshals arguments and
     keeps (Q, K, V, O, lse, sel) for the backward call.
 
-    apply(layout, Q, K, V, k, causal=True, scale=None) -> O (bf16 [B, H, L, d]);
-    the selection of the last call is left in ``MoCAttention.last_sel``."""
-
-    last_sel: Optional[torch.Tensor] = None
+    apply(layout, Q, K, V, k, causal=True, scale=None) -> O (bf16 [B, H, L, d])."""
 
     @staticmethod
     def forward(ctx, layout, Q, K, V, k, causal=True, scale=None):
@@ -360,7 +357,6 @@ class MoCAttention(torch.autograd.Function):
         O, lse, sel, _ = forward(layout, Q, K, V, k, causal, scale)
         ctx.layout, ctx.k, ctx.scale = layout, k, scale
         ctx.save_for_backward(Q, K, V, O, lse, sel)
-        MoCAttention.last_sel = sel
         return O
 
     @staticmethod

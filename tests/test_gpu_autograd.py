@@ -41,7 +41,6 @@ def test_autograd_equals_the_backward_call(which):
     dQ, dK, dV = moc.attention_bwd(lay, Q, K, V, O2, lse2, G, sel2, wl.k)
     torch.cuda.synchronize()
     assert torch.equal(O.detach().view(torch.int16), O2.view(torch.int16))
-    assert torch.equal(moc.MoCAttention.last_sel, sel2)
     for got, want in ((Qr.grad, dQ), (Kr.grad, dK), (Vr.grad, dV)):
         assert got.dtype == torch.bfloat16 and got.shape == want.shape
         assert torch.equal(got.view(torch.int16), want.view(torch.int16))
