@@ -26,10 +26,17 @@ __global__ void __launch_bounds__(32) qlist_count(int L, int C, int k, int nblk,
     __syncwarp();
     const int q0 = blk * kQlistBlock, q1 = min(L, q0 + kQlistBlock);
     const int32_t* s = sel + (size_t(bh) * L) * k;
-    for (int64_t e = int64_t(q0) * k + lane; e < int64_t(q1) * k; e += 32) {
-        const int c = s[e];
-        if (c >= C) set_error(hdr, ERR_CHECK, 3);  // not a chunk id: entry ignored
-        else if (c >= 0) atomicAdd(&cnt[c], 1);
+    constexpr int U = 4;  // entries per lane loaded per round trip
+    const int64_t e1 = int64_t(q1) * k;
+    for (int64_t e0 = int64_t(q0) * k + lane; e0 < e1; e0 += 32 * U) {
+        int cs[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) cs[u] = (e0 + 32 * u < e1) ? s[e0 + 32 * u] : -1;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (cs[u] >= C) set_error(hdr, ERR_CHECK, 3);  // not a chunk id: entry ignored
+            else if (cs[u] >= 0) atomicAdd(&cnt[cs[u]], 1);
+        }
     }
     __syncwarp();
     int32_t* out = blk_count + (size_t(bh) * nblk + blk) * C;
@@ -45,13 +52,19 @@ __global__ void __launch_bounds__(256) qlist_scan_blocks(int C, int nblk,
                                                          int32_t* __restrict__ ntile,
                                                          int32_t* __restrict__ ntile2) {
     const int bh = blockIdx.x;
+    constexpr int U = 8;  // block counts loaded per round trip
     for (int c = threadIdx.x; c < C; c += blockDim.x) {
         int32_t run = 0;
         int32_t* p = blk_count + size_t(bh) * nblk * C + c;
-        for (int b = 0; b < nblk; ++b) {
-            const int32_t v = p[size_t(b) * C];
-            p[size_t(b) * C] = run;
-            run += v;
+        for (int b0 = 0; b0 < nblk; b0 += U) {
+            int32_t v[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) v[u] = (b0 + u < nblk) ? p[size_t(b0 + u) * C] : 0;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (b0 + u < nblk) p[size_t(b0 + u) * C] = run;
+                run += v[u];
+            }
         }
         qlen[size_t(bh) * C + c] = run;
         ntile[size_t(bh) * C + c] = (run + kItemRows - 1) / kItemRows;
@@ -134,9 +147,14 @@ __global__ void __launch_bounds__(32) qlist_scatter(int L, int C, int k, int nbl
     const int q0 = blk * kQlistBlock, q1 = min(L, q0 + kQlistBlock);
     const int32_t* s = sel + (size_t(bh) * L) * k;
     const unsigned lt = (1u << lane) - 1u;
-    for (int64_t e0 = int64_t(q0) * k; e0 < int64_t(q1) * k; e0 += 32) {
+    const int64_t e1 = int64_t(q1) * k;
+    // each step's selection entry is loaded one step ahead, so the load latency
+    // overlaps the previous step's ranking and stores
+    int c_next = (int64_t(q0) * k + lane < e1) ? s[int64_t(q0) * k + lane] : -1;
+    for (int64_t e0 = int64_t(q0) * k; e0 < e1; e0 += 32) {
         const int64_t e = e0 + lane;
-        int c = (e < int64_t(q1) * k) ? s[e] : -1;
+        int c = c_next;
+        c_next = (e + 32 < e1) ? s[e + 32] : -1;
         if (c >= C) c = -1;  // reported by qlist_count
         const unsigned peers = __match_any_sync(0xffffffffu, c);
         const int rank = __popc(peers & lt);
