@@ -99,3 +99,45 @@ def test_head_split_shares_reassemble_the_whole_tensor(world):
         got = [out[r] for r in range(world)]
     want = ref.view(wl.B * wl.H, wl.L, wl.d).view(torch.int16).numpy().tobytes()
     assert all(g == want for g in got)
+
+
+def _reshard_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    sys.path.insert(0, ROOT)
+    import bench
+    import moc_workloads as W
+    wl = W.tiny().replace(B=2, H=3)
+    q, _, _ = W.make_qkv(wl)
+    full = q.view(wl.B * wl.H, wl.L, wl.d)
+    t0, t1 = bench.shard_slices(1, wl.L, world, rank)
+    s0, s1 = bench.shard_slices(wl.B, wl.H, world, rank)
+    xs = full[:, t0:t1].contiguous()            # this rank's token share of every slice
+    xh = bench.seq_to_heads(xs, wl.B * wl.H, wl.L, world, rank)
+    back = bench.heads_to_seq(xh, wl.B * wl.H, wl.L, world, rank)
+    lse = torch.arange(wl.B * wl.H * wl.L, dtype=torch.float32).view(wl.B * wl.H, wl.L)
+    lh = bench.seq_to_heads(lse[:, t0:t1].contiguous(), wl.B * wl.H, wl.L, world, rank)
+    out[rank] = (torch.equal(xh.view(torch.int16), full[s0:s1].view(torch.int16)),
+                 torch.equal(back.view(torch.int16), xs.view(torch.int16)),
+                 torch.equal(lh, lse[s0:s1]), tuple(xh.shape))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 5])
+def test_sequence_shards_reshard_to_the_head_split_and_back(world):
+    """A caller holding sequence shards (contiguous token ranges of every slice,
+    uneven at 5 ranks: 2,112 tokens, 6 slices) gets exactly the head split's
+    slices over all tokens from seq_to_heads (one all-to-all), and heads_to_seq
+    returns its own token share bit for bit; bf16 [.., L, d] and fp32 [.., L]
+    tensors both."""
+    import bench
+    port = _free_port()
+    with mp.get_context("spawn").Manager() as m:
+        out = m.dict()
+        mp.start_processes(_reshard_worker, args=(world, port, out), nprocs=world, start_method="spawn")
+        got = [out[r] for r in range(world)]
+    for r, (heads_ok, back_ok, lse_ok, shape) in enumerate(got):
+        s0, s1 = bench.shard_slices(2, 3, world, r)
+        assert heads_ok and back_ok and lse_ok, r
+        assert shape == (s1 - s0, 2112, 64)
