@@ -3,8 +3,8 @@
 // Some callers cannot hand the library a device workspace: they may not call
 // cudaMalloc at all (an inference-server plugin that is given only its input
 // and output buffers, a real-time loop that must never take the driver's
-// allocation path, which can synchronise the device, or code running under a
-// framework whose caching allocator is frozen while it records a CUDA graph).
+// allocation path, which can synchronise the device, or a library embedded in
+// a host application that budgets every device byte itself up front).
 // This entry point runs the same three stages as moc_attention_fwd (query
 // lists, attend, merge) on a fixed scratch area that lives in the library
 // itself: a file-scope static __device__ array of kStaticScratchBytes. Every

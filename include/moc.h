@@ -291,8 +291,8 @@ moc_status moc_attention_bwd(const moc_layout* layout, int B, int H, int d, cons
 
 /* moc_attention_fwd without a caller workspace, for callers that cannot
  * allocate device memory (a plugin given only its input and output buffers, a
- * real-time loop that must stay off the driver's allocation path, code running
- * while a framework's allocator is frozen for graph capture). The pages
+ * real-time loop that must stay off the driver's allocation path, a library
+ * inside a host application that budgets every device byte up front). The pages
  * describe no counterpart: this is a deployment variant of (3)-(5) above.
  * Scratch: a static 64 MiB device array inside the library, held on every GPU
  * that loads it until the process exits; nothing is allocated per call.
