@@ -240,3 +240,22 @@ def test_backward_key_blocks_agree_with_oracle_roles(wl):
     assert kt_off[0] == 0 and len(kt_off) == nkb + 1
     for x, b in enumerate(kb_order):
         assert kt_off[x + 1] - kt_off[x] == (rng_[b, 1] - rng_[b, 0] + 127) // 128
+
+
+@pytest.mark.parametrize("n_chunks,ok", [(16384, True), (16385, False)])
+def test_chunk_count_limit(n_chunks, ok):
+    """C = 16,384 chunks (the library's limit: the query-list counters of one
+    (b, h) live in shared memory) builds; one more is rejected as a bad layout.
+    One-token frames, 16 shots (the last shot takes the remainder)."""
+    per = 1024
+    ln = [1] * n_chunks
+    kind = [1] * n_chunks
+    shot = [min(i // per, 15) for i in range(n_chunks)]
+    frame = [i - shot[i] * per for i in range(n_chunks)]
+    if ok:
+        lay = moc.Layout(ln, kind, shot, frame, "shot", 0, device=-1)
+        assert lay.C == n_chunks and lay.L == n_chunks
+    else:
+        with pytest.raises(moc.MocError) as ei:
+            moc.Layout(ln, kind, shot, frame, "shot", 0, device=-1)
+        assert ei.value.status == 2

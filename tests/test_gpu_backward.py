@@ -96,6 +96,18 @@ def test_small_ragged_scene_d128():
     _full_case(wl)
 
 
+def test_largest_k_every_row_and_key():
+    """k = 31 (the largest top-k): 32 partial dQ slots a row, 31 of them routed;
+    three shots of 16 sub-chunks of 20-80 tokens, every row and key."""
+    rng = np.random.default_rng(7)
+    segs = []
+    for s_ in range(3):
+        segs.append(W.Segment(16, W.CAPTION, s_, -1))
+        for f in range(16):
+            segs.append(W.Segment(int(rng.integers(20, 81)), W.VIDEO, s_, f))
+    _full_case(W.custom("manychunks", 1, 2, 128, segs, "shot", 0, True, 31, 33, "frame"))
+
+
 def test_backward_is_deterministic():
     wl = W.tiny()
     Q, K, V = W.make_qkv(wl)

@@ -84,6 +84,18 @@ def test_small_ragged_scene_every_row(k, anchor):
     _check(_ragsmall(k=k, anchor=anchor))
 
 
+def test_largest_k_every_row():
+    """k = 31: 32 partial slots a row; three shots of 16 sub-chunks of 20-140
+    tokens (the last shot's queries pick 31 of 32 candidates)."""
+    rng = np.random.default_rng(7)
+    segs = []
+    for s_ in range(3):
+        segs.append(W.Segment(16, W.CAPTION, s_, -1))
+        for f in range(16):
+            segs.append(W.Segment(int(rng.integers(20, 141)), W.VIDEO, s_, f))
+    _check(W.custom("manychunks", 1, 2, 128, segs, "shot", 0, True, 31, 33, "frame"))
+
+
 def test_non_causal_scene_every_row():
     """Routing over earlier and later chunks: longer query lists per chunk."""
     wl = _ragsmall(k=4)

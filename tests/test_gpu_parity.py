@@ -73,6 +73,29 @@ def test_tiny_all_rows():
     assert res["mismatch"] == 0
 
 
+def _many_chunk_scene(d: int, k: int):
+    """Three shots of 16 sub-chunks (20-140 tokens each) with a 16-token caption
+    before each shot: queries of the last shot have 32 routing candidates."""
+    rng = np.random.default_rng(7)
+    segs = []
+    for s_ in range(3):
+        segs.append(W.Segment(16, W.CAPTION, s_, -1))
+        for f in range(16):
+            segs.append(W.Segment(int(rng.integers(20, 141)), W.VIDEO, s_, f))
+    return W.custom("manychunks", 1, 2, d, segs, "shot", 0, True, k, 33, "frame")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_largest_k_every_row(d):
+    """k = 31, the largest top-k the library takes (1 + k partial slots a row fill
+    one warp; query-list entries keep the slot in 5 bits): every row against the
+    oracle, with lists of 32 candidates (31 picked), 16 (all picked, 15 pads) and
+    none; then chunk anchors without the causal mask (47 candidates a query)."""
+    wl = _many_chunk_scene(d, 31)
+    _check_full(wl)
+    _check_full(wl.replace(anchor="chunk", causal=False))
+
+
 @pytest.mark.parametrize("k", [0, 1, 3, 8])
 def test_tiny_k_edge_cases(k):
     """k = 0 (anchors only), k > |candidates| (shot 1 has 4): padding with -1."""
