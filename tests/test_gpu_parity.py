@@ -3,6 +3,7 @@
 Inputs are the seeded synthetic workloads of ``moc_workloads``; the same CPU
 bytes feed the oracle and the GPU. Tolerances are in ``tests/parity.py``.
 """
+import ctypes
 import math
 import time
 
@@ -94,6 +95,27 @@ def test_largest_k_every_row(d):
     wl = _many_chunk_scene(d, 31)
     _check_full(wl)
     _check_full(wl.replace(anchor="chunk", causal=False))
+
+
+def test_largest_slice_count():
+    """B * H = 65,535 (b, h) slices, the library's limit (slices index the second
+    launch dimension of the pool and query-list kernels): an 80-token scene with
+    every stage launched over all slices; the first two and the last slice are
+    generated and checked against the oracle on every row (the rest are zero
+    inputs). One slice more is rejected before any launch."""
+    segs = [W.Segment(16, W.CAPTION, 0, -1)]
+    for s_ in range(2):
+        for f in range(2):
+            segs.append(W.Segment(16, W.VIDEO, s_, f))
+    wl = W.custom("manyslices", 1, 65535, 64, segs, "shot", 0, True, 1, 35, "frame")
+    _check_full(wl, heads=[(0, 0), (0, 1), (0, 65534)])
+    lay = moc.Layout.from_workload(wl)
+    p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    lib = moc.lib()
+    assert lib.moc_pool_keys(lay.handle, 1, 65536, 64, p, p, moc._stream()) == 1
+    assert lib.moc_route(lay.handle, 2, 32768, 64, p, p, 1, 1, p, moc._stream()) == 1
+    assert lib.moc_attention_fwd(lay.handle, 1, 65536, 64, p, p, p, p, 1, 0.125, p, None, p,
+                                 1 << 30, moc._stream()) == 1
 
 
 @pytest.mark.parametrize("k", [0, 1, 3, 8])
