@@ -430,7 +430,9 @@ def run_ours(args):
         "warmup": args.warmup,
         "ms_per_step": ms_per_step,
         "higher_is_better": True,
-        "scaling": "strong" if shard == "heads" else "weak",
+        # the series the same command forms over N: --shard heads splits one scene
+        # (total work fixed, also at N = 1), --shard replicas adds a scene per rank
+        "scaling": "strong" if args.shard == "heads" else "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) + per-shot/per-frame mean offsets; no dataset)",
@@ -782,7 +784,8 @@ def run_reference(args):
               f"before timing ({t_pool:.3f} s)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": ws_, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": step_s * 1e3, "higher_is_better": True,
+            "scaling": "strong" if args.shard == "heads" else "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": workload_string(wl, lay.C),
                        "tokens_per_step": tokens_per_step},
