@@ -28,11 +28,12 @@
 //   warps 0 .. 4*NWG-1: selection warpgroups taking tiles round robin; one
 //          thread per query row (= TMEM lane) reads its scores from TMEM and
 //          keeps a sorted top-KMAX list in registers with a branch-free
-//          insertion network (candidates come in ascending id, so a strict
-//          ">" orders ties by lower chunk id), writing the first k entries
-//          (-1 padded) after the tile's last slice. The network is a chain of
-//          dependent compare/select steps per row, so more warpgroups (more
-//          rows in flight per scheduler) hide its latency.
+//          insertion network over packed score / position keys (lists of up
+//          to 511 entries; candidates come in ascending id, so equal keys
+//          order by lower chunk id), writing the first k entries (-1 padded)
+//          after the tile's last slice. The network is a chain of dependent
+//          max / min steps per row, so more warpgroups (more rows in flight
+//          per scheduler) hide its latency.
 // Tiles without candidates (caption groups, the first shot) are written as -1
 // rows by their selection warpgroup and skip the other roles. Waits are
 // bounded as in the attention kernel; a timeout is recorded in the layout's
@@ -122,12 +123,14 @@ __device__ __forceinline__ void topk_push(float (&ts)[KMAX], int (&tj)[KMAX], fl
     }
 }
 
-// For k > 4, and for candidate lists longer than 128 entries: an order-preserving
-// 32-bit key of a score with the candidate's position in its 9 low bits (larger
-// score first, then lower position), so an insertion step is one max and one min. The score keeps all but the 9 lowest
-// bits of its order-preserving integer image: scores closer than 2^-14 of their
-// magnitude compare equal and go by position (chunk id), a gap well inside the
-// 1e-4 relative near-tie tolerance that routing is checked with.
+// For candidate lists of up to 511 entries (positions fit 9 bits): an
+// order-preserving 32-bit key of a score with the candidate's position in its 9
+// low bits (larger score first, then lower position), so an insertion step is one
+// max and one min instead of a compare, a max / min pair and two selects. The
+// score keeps all but the 9 lowest bits of its order-preserving integer image:
+// scores closer than 2^-14 of their magnitude compare equal and go by position
+// (chunk id), a gap well inside the 1e-4 relative near-tie tolerance that routing
+// is checked with. (Eight-shot scene, k = 3: 0.383 -> 0.359 ms.)
 __device__ __forceinline__ uint32_t pack_key(float s, int pos) {
     const uint32_t u = __float_as_uint(s);
     const uint32_t o = u ^ (uint32_t(int32_t(u) >> 31) | 0x80000000u);
@@ -518,12 +521,12 @@ cudaError_t launch_dk(const DevLayout& dv, int BH, int64_t rtiles, const void* Q
                       int causal, int max_cand, const uint64_t* seg_mask, int32_t* sel, cudaStream_t s) {
     if constexpr (RWarps<KMAX>::kSlice <= 128) {
         if (max_cand <= 128)
-            return launch_cfg<D, KMAX, 128, 5, (KMAX >= 8)>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
+            return launch_cfg<D, KMAX, 128, 5, true>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
     }
     // lists of up to 320 entries fit one operand block beside a 2-stage ring, so a
-    // group's block is built once instead of once per tile and block; with lists this
-    // long (and for k > 4) the selection uses packed score / position keys (positions
-    // below 512): it is the kernel's main cost there (ragged k = 2: 1.44 -> 0.80 ms)
+    // group's block is built once instead of once per tile and block; the selection
+    // uses packed score / position keys (positions below 512): it is the kernel's main
+    // cost with lists this long (ragged k = 2: 1.44 -> 0.80 ms)
     if constexpr (KMAX >= 8) {
         if (max_cand <= 320)
             return launch_cfg<D, KMAX, 320, 2, true>(dv, BH, rtiles, Q, Kbar, k, causal, seg_mask, sel, s);
