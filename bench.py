@@ -88,17 +88,30 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.lines = []
+        self.skip = 0
 
     def start(self):
+        """Start sampling every 100 ms and return once the first sample is in
+        (nvidia-smi takes a while to start); mark() then sets where the counted
+        samples begin."""
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
         except OSError:
             self.proc = None
+            return
+        t0 = time.time()
+        while not self.lines and time.time() - t0 < 5.0 and self.proc.poll() is None:
+            time.sleep(0.01)
+        self.skip = len(self.lines)
+
+    def mark(self):
+        """Count only the samples taken from now on (the timed region)."""
+        self.skip = len(self.lines)
 
     def _read(self):
         for line in self.proc.stdout:
@@ -115,7 +128,8 @@ class ClockSampler:
         self.t.join(timeout=2)
         sm, mx, reasons, power = [], None, set(), []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        lines = self.lines[self.skip:] or self.lines
+        for ln in lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -337,6 +351,10 @@ def run_ours(args):
         moc.merge(lay, sel, k, ws, O, lse)
         if ev: ev[5].record(stream)
 
+    # clocks are sampled from before the warm-up steps (the sampler takes a while to
+    # start) and counted from the start of the timed region
+    clocks = ClockSampler(local)
+    clocks.start()
     for _ in range(args.warmup):
         step()
     moc.check_device_error(ws)
@@ -349,10 +367,9 @@ def run_ours(args):
             torch.distributed.barrier()
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(args.steps)]
-    clocks = ClockSampler(local)
     barrier()
     torch.cuda.synchronize()
-    clocks.start()
+    clocks.mark()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
