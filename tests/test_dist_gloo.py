@@ -1,6 +1,8 @@
-"""Multi-rank host logic of bench.py on CPU (gloo, world size 2): each rank
-gets an independent scene, times are reduced with max over ranks, and the
-reference arm prints one line from rank 0 while the other rank exits 0."""
+"""Multi-rank host logic on CPU (gloo): in bench.py each replica rank gets an
+independent scene, times are reduced with max over ranks, and the reference arm
+prints one line from rank 0 while the other rank exits 0; the head split, the
+all-gather of its shares and the sequence re-sharding of
+chunk_routed_sparse_b200.sharding cover every slice and token exactly once."""
 import json
 import os
 import socket
@@ -60,10 +62,10 @@ def test_reference_arm_under_torchrun_prints_once():
 
 
 def test_head_split_covers_every_slice_once_and_balanced():
-    import bench
+    from chunk_routed_sparse_b200 import sharding
     for B, H in [(1, 24), (2, 24), (1, 5), (3, 7)]:
         for world in (1, 2, 3, 4, 8):
-            shares = [bench.shard_slices(B, H, world, r) for r in range(world)]
+            shares = [sharding.shard_slices(B, H, world, r) for r in range(world)]
             covered = [i for a, b in shares for i in range(a, b)]
             assert covered == list(range(B * H)), (B, H, world)
             sizes = [b - a for a, b in shares]
@@ -74,12 +76,12 @@ def _gather_worker(rank, world, port, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     sys.path.insert(0, ROOT)
-    import bench
     import moc_workloads as W
+    from chunk_routed_sparse_b200 import sharding
     wl = W.tiny().replace(B=2, H=3)            # 6 slices over `world` ranks
-    s0, s1 = bench.shard_slices(wl.B, wl.H, world, rank)
+    s0, s1 = sharding.shard_slices(wl.B, wl.H, world, rank)
     q, _, _ = W.make_qkv_slices(wl, s0, s1)    # this rank's share of the scene's Q
-    full = bench.gather_slices(q.view(s1 - s0, wl.L, wl.d), wl.B * wl.H, world)
+    full = sharding.gather_slices(q.view(s1 - s0, wl.L, wl.d), wl.B * wl.H, world)
     out[rank] = full.view(torch.int16).numpy().tobytes()
     dist.barrier()
     dist.destroy_process_group()
@@ -105,18 +107,18 @@ def _reshard_worker(rank, world, port, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     sys.path.insert(0, ROOT)
-    import bench
     import moc_workloads as W
+    from chunk_routed_sparse_b200 import sharding
     wl = W.tiny().replace(B=2, H=3)
     q, _, _ = W.make_qkv(wl)
     full = q.view(wl.B * wl.H, wl.L, wl.d)
-    t0, t1 = bench.shard_slices(1, wl.L, world, rank)
-    s0, s1 = bench.shard_slices(wl.B, wl.H, world, rank)
+    t0, t1 = sharding.shard_slices(1, wl.L, world, rank)
+    s0, s1 = sharding.shard_slices(wl.B, wl.H, world, rank)
     xs = full[:, t0:t1].contiguous()            # this rank's token share of every slice
-    xh = bench.seq_to_heads(xs, wl.B * wl.H, wl.L, world, rank)
-    back = bench.heads_to_seq(xh, wl.B * wl.H, wl.L, world, rank)
+    xh = sharding.seq_to_heads(xs, wl.B * wl.H, wl.L, world, rank)
+    back = sharding.heads_to_seq(xh, wl.B * wl.H, wl.L, world, rank)
     lse = torch.arange(wl.B * wl.H * wl.L, dtype=torch.float32).view(wl.B * wl.H, wl.L)
-    lh = bench.seq_to_heads(lse[:, t0:t1].contiguous(), wl.B * wl.H, wl.L, world, rank)
+    lh = sharding.seq_to_heads(lse[:, t0:t1].contiguous(), wl.B * wl.H, wl.L, world, rank)
     out[rank] = (torch.equal(xh.view(torch.int16), full[s0:s1].view(torch.int16)),
                  torch.equal(back.view(torch.int16), xs.view(torch.int16)),
                  torch.equal(lh, lse[s0:s1]), tuple(xh.shape))
@@ -131,13 +133,13 @@ def test_sequence_shards_reshard_to_the_head_split_and_back(world):
     slices over all tokens from seq_to_heads (one all-to-all), and heads_to_seq
     returns its own token share bit for bit; bf16 [.., L, d] and fp32 [.., L]
     tensors both."""
-    import bench
+    from chunk_routed_sparse_b200 import sharding
     port = _free_port()
     with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.start_processes(_reshard_worker, args=(world, port, out), nprocs=world, start_method="spawn")
         got = [out[r] for r in range(world)]
     for r, (heads_ok, back_ok, lse_ok, shape) in enumerate(got):
-        s0, s1 = bench.shard_slices(2, 3, world, r)
+        s0, s1 = sharding.shard_slices(2, 3, world, r)
         assert heads_ok and back_ok and lse_ok, r
         assert shape == (s1 - s0, 2112, 64)
